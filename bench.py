@@ -1,0 +1,576 @@
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of one attention layer over a batch of sequences:
+the host block manager reserves every sequence's next slot (copy-on-write
+pairs if any -> copy_blocks), reshape_and_cache writes the new K/V, and
+paged decode attention (+ the split-context merge) reads every cached token
+of every sequence through the block tables.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa8b]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  `value` is the decode attention's algorithmic
+HBM bytes (every K/V element of every cached token read once, plus the block
+table entries used) divided by the device-timed step; `e2e` is the same
+metric through the public API from pinned host buffers, with the block
+manager, the host->device copy of the step's inputs and the device->host copy
+of its output inside the timed region.  Inputs are larger than L2, so no L2
+flush is needed between steps.  Data are synthetic (seeded, see workloads.py).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+WORKLOADS = {
+    "gqa8b": "GQA 8B-class paged decode: 256 seqs, 32 q / 8 kv heads, head_dim 128, block 16, "
+             "bf16 KV, lognormal context lengths (median 512, clip 16..4096), shuffled blocks",
+    "13b": "13B-class paged decode: 64 seqs, 40 q = 40 kv heads, head_dim 128, block 16, fp16 KV, "
+           "context lengths uniform 1..2048, shuffled blocks",
+    "long": "long-context paged decode: 8 seqs, 64 q / 8 kv heads, head_dim 128, block 16, bf16, "
+            "context lengths uniform 16384..32768, peaked softmax",
+    "long32": "long-context paged decode, block 32",
+}
+METRIC = "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_attention_gqa8b.md")
+KERNEL_SOURCES = ["paged_kv_cache_414_b200/csrc/decode_attention.cuh",
+                  "paged_kv_cache_414_b200/csrc/pa_device.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha():
+        return None
+    return float(m_tr.group(1))
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_cores_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([int(x.get("num_threads", 1)) for x in threadpool_info()] + [1])
+        return n
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- workload
+
+class Workload:
+    """A decode batch plus K+W steps of block-manager output prepared ahead."""
+
+    def __init__(self, name: str, device, seed_offset: int, steps_total: int):
+        import torch
+        self.name = name
+        sh = W.SHAPES[name]
+        self.shape = sh
+        rng = np.random.default_rng(W.SEEDS[name] + 1000 * seed_offset)
+        lens = {"gqa8b": W.lens_gqa8b, "13b": W.lens_13b}.get(name, W.lens_long)(rng)
+        B = sh.block_size
+        grow = math.ceil(steps_total / B) + 1
+        need = sum(math.ceil(int(L) / B) + grow for L in lens)
+        maxb = max(math.ceil((int(L) + steps_total) / B) for L in lens)
+        self.batch = W.make_decode_batch(sh, lens, W.SEEDS[name] + 1000 * seed_offset,
+                                         device=device, num_blocks=int(need * 1.1),
+                                         max_blocks_per_seq=maxb, rng=rng)
+        self.lens0 = lens.astype(np.int64)
+        self.maxb = maxb
+        self.S = len(lens)
+        self.device = device
+        self.scale = 1.0 / math.sqrt(sh.head_dim)
+        self.elem = 2
+
+    def bytes_per_step(self, step: int) -> int:
+        from paged_kv_cache_414_b200 import decode_bytes
+        return decode_bytes(self.lens0 + step, self.shape.num_kv_heads, self.shape.head_dim,
+                            self.shape.block_size, self.elem)
+
+    def new_manager(self, pa):
+        bm = pa.BlockManager(self.batch.num_blocks, self.shape.block_size, self.batch.free_order)
+        for s in range(self.S):
+            bm.allocate(s, int(self.lens0[s]) - 1)
+        return bm
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_b200(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_414_b200 import build as pbuild
+    pbuild.build()
+    import paged_kv_cache_414_b200 as pa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    K, Wm = args.steps, args.warmup
+    wl = Workload(args.workload, dev, rank, K + Wm + 1)
+    sh = wl.shape
+    B = sh.block_size
+    S = wl.S
+    b = wl.batch
+    stream = torch.cuda.current_stream()
+
+    # block manager output for every step, prepared ahead (device-resident arm)
+    bm = wl.new_manager(pa)
+    seqs = np.arange(S)
+    d_slots, d_tables, d_lens, d_pairs = [], [], [], []
+    for step in range(K + Wm):
+        slots, pairs = bm.append_slots(seqs)
+        tables, lens = bm.block_tables(seqs, wl.maxb)
+        d_slots.append(torch.as_tensor(slots, device=dev))
+        d_tables.append(torch.as_tensor(tables, device=dev))
+        d_lens.append(torch.as_tensor(lens, device=dev))
+        d_pairs.append(torch.as_tensor(pairs, device=dev) if len(pairs) else None)
+    bm.close()
+    maxctx = wl.maxb * B
+    ws = pa.alloc_workspace(S, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, B, maxctx, dev)
+    out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+    launches_per_step = 3   # reshape_and_cache, decode attention, split merge
+
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def step(i, timed_idx=None):
+        if d_pairs[i] is not None:
+            pa.pa_copy_blocks(b.k_cache, b.v_cache, d_pairs[i])
+        pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, d_slots[i])
+        if timed_idx is not None:
+            ev_a[timed_idx].record(stream)
+        pa.pa_paged_decode_attention(out, b.q, b.k_cache, b.v_cache, d_tables[i], d_lens[i],
+                                     wl.scale, sh.num_kv_heads, max_context_len=maxctx,
+                                     workspace=ws)
+        if timed_idx is not None:
+            ev_b[timed_idx].record(stream)
+
+    for i in range(Wm):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" in os.environ
+                          else local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0.record(stream)
+    for k in range(K):
+        step(Wm + k, k)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    flags = pa.pa_device_error()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = [ev_a[k].elapsed_time(ev_b[k]) for k in range(K)]
+    bytes_steps = [wl.bytes_per_step(Wm + k) for k in range(K)]
+    my_bytes = float(sum(bytes_steps))
+
+    def reduce_max(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def reduce_sum(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    ms_max = reduce_max(ms_total)
+    all_bytes = reduce_sum(my_bytes)
+    value = all_bytes / (ms_max * 1e-3) / 1e9
+    tokens_per_s = reduce_sum(float(S * K)) / (ms_max * 1e-3)
+
+    # roofline of the decode attention call (attention + merge kernels)
+    attn_avg_ms = float(np.mean(attn_ms))
+    bytes_launch = float(np.mean(bytes_steps))
+    achieved = bytes_launch / (attn_avg_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    traffic = profiled_traffic()
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": Wm,
+            "ms_per_step": round(ms_max / K, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": sh.dtype,
+            "data": "synthetic",
+            "config": {
+                "workload": f"{args.workload}: {WORKLOADS[args.workload]}",
+                "num_seqs_per_gpu": S,
+                "num_q_heads": sh.num_q_heads,
+                "num_kv_heads": sh.num_kv_heads,
+                "head_dim": sh.head_dim,
+                "block_size": B,
+                "mean_context_len": float(np.mean(wl.lens0)) + Wm + (K - 1) / 2,
+                "parallelism": f"dp{world} (independent batches, no collective on the data path)",
+                "l2": "inputs larger than L2: %.2f GB of KV read per step, no flush" % (bytes_launch / 1e9),
+                "step": "host block manager (prepared ahead) -> reshape_and_cache -> paged decode attention + split merge",
+            },
+            "pct_of_measured_hbm_peak": round(100.0 * value / peak / world, 2),
+            "pct_of_nominal_8tbs": round(100.0 * value / 8000.0 / world, 2),
+            "decode_tokens_per_s": round(tokens_per_s, 1),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "pa_paged_decode_attention (paged_decode_kernel + paged_decode_merge_kernel)",
+                "achieved": round(achieved, 2),
+                "peak": peak,
+                "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6650 GB/s",
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": traffic,
+                "bytes_per_launch": bytes_launch,
+                "avg_launch_ms": round(attn_avg_ms, 5),
+            },
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": launches_per_step * K,
+            "device_error_flags": flags,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
+    """Same metric through the public API from pinned host buffers: block
+    manager on the host, H2D of the step's inputs, kernels, D2H of the output."""
+    import torch
+    import torch.distributed as dist
+    sh = wl.shape
+    S, B = wl.S, sh.block_size
+    b = wl.batch
+    seqs = np.arange(S)
+    bm = wl.new_manager(pa)
+    # host copies of the step's inputs (values reused each step)
+    h_q = [b.q.cpu().pin_memory() for _ in range(2)]
+    h_k = [b.k_new.cpu().pin_memory() for _ in range(2)]
+    h_v = [b.v_new.cpu().pin_memory() for _ in range(2)]
+    h_slots = [torch.empty(S, dtype=torch.int64).pin_memory() for _ in range(2)]
+    h_tables = [torch.empty(S, wl.maxb, dtype=torch.int32).pin_memory() for _ in range(2)]
+    h_lens = [torch.empty(S, dtype=torch.int32).pin_memory() for _ in range(2)]
+    h_out = [torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32).pin_memory()
+             for _ in range(2)]
+    d_q = torch.empty_like(b.q)
+    d_k = torch.empty_like(b.k_new)
+    d_v = torch.empty_like(b.v_new)
+    d_slots = torch.empty(S, dtype=torch.int64, device=dev)
+    d_tables = torch.empty(S, wl.maxb, dtype=torch.int32, device=dev)
+    d_lens = torch.empty(S, dtype=torch.int32, device=dev)
+    d_out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+    maxctx = wl.maxb * B
+    ws = pa.alloc_workspace(S, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, B, maxctx, dev)
+    done = [None, None]
+    h2d = sum(t[0].numel() * t[0].element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_lens))
+    d2h = h_out[0].numel() * 4
+
+    def one(i):
+        j = i % 2
+        if done[j] is not None:
+            done[j].synchronize()          # buffers of step i-2 are free again
+        slots, pairs = bm.append_slots(seqs)
+        h_slots[j].numpy()[:] = slots
+        tables, lens = bm.block_tables(seqs, wl.maxb)
+        h_tables[j].numpy()[:] = tables
+        h_lens[j].numpy()[:] = lens
+        d_q.copy_(h_q[j], non_blocking=True)
+        d_k.copy_(h_k[j], non_blocking=True)
+        d_v.copy_(h_v[j], non_blocking=True)
+        d_slots.copy_(h_slots[j], non_blocking=True)
+        d_tables.copy_(h_tables[j], non_blocking=True)
+        d_lens.copy_(h_lens[j], non_blocking=True)
+        if len(pairs):
+            pa.pa_copy_blocks(b.k_cache, b.v_cache, torch.as_tensor(pairs).to(dev, non_blocking=True))
+        pa.pa_reshape_and_cache(d_k, d_v, b.k_cache, b.v_cache, d_slots)
+        pa.pa_paged_decode_attention(d_out, d_q, b.k_cache, b.v_cache, d_tables, d_lens,
+                                     wl.scale, sh.num_kv_heads, max_context_len=maxctx,
+                                     workspace=ws)
+        h_out[j].copy_(d_out, non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record()
+        done[j] = ev
+
+    for i in range(Wm):
+        one(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(Wm, Wm + K):
+        one(i)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    bm.close()
+    dt_max = reduce_max(dt)
+    bytes_all = reduce_sum(float(sum(wl.bytes_per_step(i) for i in range(Wm, Wm + K))))
+    return {"value": round(bytes_all / dt_max / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(dt_max * 1e3 / K, 4),
+            "timing": "host wall clock, synchronize on both sides, max over ranks"}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_step_sample(wl, step: int, seqs):
+    """The oracle's decode step for some sequences: its own block manager's
+    slots, its own cache write, its own attention.  Returns (out, bytes)."""
+    from oracle import attention as OA
+    from oracle import cache_ops as OC
+    from oracle.block_manager import BlockManager as OracleBM
+    sh = wl.shape
+    B = sh.block_size
+    b = wl.batch
+    bm = OracleBM(b.num_blocks, B, b.free_order)
+    for s in range(wl.S):
+        bm.allocate(s, int(wl.lens0[s]) - 1 + step)
+    slots = [bm.append_slot(s)[0] for s in range(wl.S)]
+    need = sorted({x for s in seqs for x in bm.block_table(s)})
+    remap = {x: i for i, x in enumerate(need)}
+    import torch
+    idx = torch.as_tensor(need, device=b.k_cache.device)
+    kb = W.bits(b.k_cache.index_select(0, idx))
+    vb = W.bits(b.v_cache.index_select(0, idx))
+    qb, knb, vnb = W.bits(b.q)[seqs], W.bits(b.k_new)[seqs], W.bits(b.v_new)[seqs]
+    sub = [remap[slots[s] // B] * B + slots[s] % B for s in seqs]
+    t0 = time.perf_counter()
+    OC.reshape_and_cache(knb, vnb, kb, vb, np.array(sub), B)
+    tabs = np.full((len(seqs), wl.maxb), -1, dtype=np.int64)
+    lens = np.zeros(len(seqs), dtype=np.int64)
+    for i, s in enumerate(seqs):
+        t = [remap[x] for x in bm.block_table(s)]
+        tabs[i, :len(t)] = t
+        lens[i] = bm.seq_len(s)
+    OA.paged_decode_attention(qb, kb, vb, tabs, lens, wl.scale, sh.num_kv_heads, B, sh.dtype)
+    dt = time.perf_counter() - t0
+    from paged_kv_cache_414_b200 import decode_bytes
+    return dt, decode_bytes(lens, sh.num_kv_heads, sh.head_dim, B, 2)
+
+
+def cpu_baseline(wl, seconds: float):
+    rng = np.random.default_rng(0)
+    order = rng.permutation(wl.S)
+    spent, nbytes, done = 0.0, 0, []
+    for s in order:
+        dt, nb = oracle_step_sample(wl, 0, [int(s)])
+        spent += dt
+        nbytes += nb
+        done.append(int(s))
+        if spent >= seconds:
+            break
+    return {"value": round(nbytes / spent / 1e9, 4), "unit": "GB/s", "cores": cpu_cores_used(),
+            "kind": "oracle",
+            "sample": f"{len(done)} of {wl.S} sequences of one step of the same workload "
+                      f"(oracle cache write + fp64 attention), {spent:.1f} s of CPU work"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, on bounded samples of the same workload."""
+    if rank != 0:
+        return
+    import torch
+    K, Wm = args.steps, args.warmup
+    wl = Workload(args.workload, "cpu", 0, K + Wm + 1)
+    per_step_budget = max(0.5, min(6.0, 150.0 / max(1, K + Wm)))
+    rng = np.random.default_rng(1)
+    order = rng.permutation(wl.S).tolist()
+    # size one step's sample so it takes about per_step_budget seconds
+    dt, _ = oracle_step_sample(wl, 0, order[:1])
+    nseq = max(1, min(wl.S, int(per_step_budget / max(dt, 1e-3))))
+    times, nbytes = [], []
+    for i in range(Wm + K):
+        seqs = [order[(i * nseq + j) % wl.S] for j in range(nseq)]
+        dt, nb = oracle_step_sample(wl, i, seqs)
+        if i >= Wm:
+            times.append(dt)
+            nbytes.append(nb)
+    value = sum(nbytes) / sum(times) / 1e9
+    sh = wl.shape
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": round(1e3 * sum(times) / K, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}",
+                   "num_seqs_per_gpu": wl.S, "num_q_heads": sh.num_q_heads,
+                   "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
+                   "block_size": sh.block_size, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_cores_used(),
+                         "kind": "oracle",
+                         "sample": f"{nseq} of {wl.S} sequences per step (oracle cache write + "
+                                   f"fp64 attention)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_b200(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

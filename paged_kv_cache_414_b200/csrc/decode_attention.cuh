@@ -1,0 +1,814 @@
+// PagedAttention decode for sm_100a.
+//
+// What is computed ("Why OS Virtual Memory Paging Saved LLM Inference: The
+// vLLM Breakthrough", section 2 "The PagedAttention Architecture"; "Can OS
+// paging techniques reduce LLM serving memory waste?", second paragraph): for
+// the newly generated token of every sequence, attention over the sequence's
+// K/V, which lives in fixed-size blocks anywhere in a physical pool and is
+// found through the sequence's block table, computed block by block.
+//
+// Work decomposition (a design for this GPU, not from the pages).  A "tile"
+// is one (sequence s, kv head h, logical block j): B tokens of K and of V,
+// B*D*2 bytes each.  Tiles are numbered in (s, h, j) order; the run of tiles
+// of one (s, h) is a "segment".  The U tiles are cut into W equal contiguous
+// ranges, one per warp of a grid that fills every SM, so every warp streams
+// the same number of bytes whatever the length mix.  A warp keeps one online
+// softmax state per segment; a segment that lies wholly inside one warp's
+// range is written to `out` directly, a segment cut by range boundaries
+// leaves one (max, sum, accumulator) partial per warp that touched it and a
+// second kernel merges them (split context).
+//
+// Data movement.  Each warp owns a ring of `nstage` shared-memory stages and
+// issues its own copies: one 2-D TMA box per 64 head-dim columns of the K
+// tile and of the V tile (128-byte swizzle, so the tensor-core fragment loads
+// below are bank-conflict free), plus a 1-D bulk copy of the G query rows at
+// the start of each segment.  Completion is counted in bytes on one mbarrier
+// per stage; every wait is bounded in time.  Block ids are prefetched for up
+// to 32 tiles ahead, one per lane.
+//
+// Arithmetic.  G = 1 (no grouped heads): fp32 FMA on CUDA cores, two lanes
+// per token for q.K and one lane per 4 (or 2) head-dim columns for P.V.
+// G >= 2: the G query heads of a group share every K/V tile, so q.K^T and
+// P.V are small dense contractions: warp-level tensor-core MMA (m16n8k16,
+// fp32 accumulate) with tokens as the M dimension of S^T = K Q^T and head-dim
+// as the M dimension of O^T = V^T P^T; P is re-laid from accumulator to
+// operand layout with movmatrix and fed as a hi + lo pair of 16-bit values so
+// the product keeps ~fp32 accuracy.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a copy never takes this long
+constexpr uint64_t kDrainLimitNs = 20000000ull;    // 20 ms to drain after a time-out
+constexpr int kMetaWords = 8;                      // int64 words per warp descriptor
+
+// Tile flags.
+enum : int {
+  TF_FIRST = 1,   // first tile of a segment in this warp's range
+  TF_LAST = 2,    // last tile of a segment in this warp's range
+  TF_J0 = 4,      // logical block 0 of the segment
+  TF_JEND = 8,    // last logical block of the segment
+  TF_SKIP = 16,   // block id out of range: no data, contributes nothing
+};
+
+struct TileInfo {
+  int s, h, j, valid, flags, pad0, pad1, pad2;
+};
+
+struct DecodeParams {
+  float *out;
+  const uint8_t *q;
+  const int32_t *block_tables;
+  const int32_t *context_lens;
+  int64_t *meta;       // [w_total][kMetaWords]
+  float *part_ml;      // [2 * w_total][G][2]   (max in log2 units, sum)
+  float *part_o;       // [2 * w_total][G][D]
+  float scale_log2;    // scale * log2(e)
+  int num_seqs, num_q_heads, num_kv_heads, group;
+  int max_blocks, num_blocks;
+  int nstage;
+  int min_tiles;       // fewest tiles a warp is given
+};
+
+__device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+// Number of blocks of sequence s, with the length clamped into the table.
+template <int B>
+__device__ __forceinline__ int seq_blocks(const DecodeParams &p, int s, bool report) {
+  int L = __ldg(p.context_lens + s);
+  const int cap = p.max_blocks * B;
+  if (L < 0 || L > cap) {
+    if (report) flag_error(PA_DEVERR_CONTEXT_LEN);
+    L = L < 0 ? 0 : cap;
+  }
+  return ceil_div_i(L, B);
+}
+
+template <int B>
+__device__ __forceinline__ int seq_len_clamped(const DecodeParams &p, int s) {
+  int L = __ldg(p.context_lens + s);
+  const int cap = p.max_blocks * B;
+  return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// Smem byte offset of (row r, 16-byte chunk c of head-dim box `box`) inside a
+// K or V tile laid out as D/64 boxes of [B rows][128 bytes] with the 128-byte
+// swizzle (chunk index XOR row % 8).
+template <int B>
+__device__ __forceinline__ uint32_t swz(int box, int r, int c) {
+  return (uint32_t)(box * (B * 128) + r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// ============================================================================
+// G >= 2: tensor-core path.  NT = number of 8-wide head tiles (G <= 8*NT).
+// ============================================================================
+template <typename T, int D, int B, int NT>
+struct MmaPath {
+  static constexpr int KT = D / 16;   // k-steps of q.K^T, m-tiles of P.V
+  static constexpr int MT = B / 16;   // token tiles per block
+  float o[KT][NT][4];
+  float m[NT][2];
+  float l[NT][2];
+  uint32_t qf[KT][NT][2];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int a = 0; a < KT; ++a)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) o[a][n][r] = 0.f;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        m[n][c] = -INFINITY;
+        l[n][c] = 0.f;
+      }
+  }
+
+  // B-operand fragments of Q^T from the staged query rows [G][D].
+  __device__ __forceinline__ void load_q(const uint8_t *qs, int G, int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int head = n * 8 + g;
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk) {
+        if (head < G) {
+          const uint8_t *row = qs + head * (D * 2) + (kk * 16 + tig * 2) * 2;
+          qf[kk][n][0] = *reinterpret_cast<const uint32_t *>(row);
+          qf[kk][n][1] = *reinterpret_cast<const uint32_t *>(row + 16);
+        } else {
+          qf[kk][n][0] = 0u;
+          qf[kk][n][1] = 0u;
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void tile(uint32_t kb, uint32_t vb, int valid, float scale_log2,
+                                       int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+    const int mi = lane >> 3, ri = lane & 7;
+    float sc[MT][NT][4];
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sc[t][n][r] = 0.f;
+
+    // S^T[token][head] = sum_d K[token][d] Q[head][d]
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const int row = t * 16 + (mi & 1) * 8 + ri;
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk) {
+        const int dim = kk * 16 + (mi >> 1) * 8;
+        uint32_t a[4];
+        ldmatrix_x4(a, kb + swz<B>(dim >> 6, row, (dim & 63) >> 3));
+#pragma unroll
+        for (int n = 0; n < NT; ++n) Mma<T>::run(sc[t][n], a, qf[kk][n][0], qf[kk][n][1]);
+      }
+    }
+
+    // scale, mask the tokens past the sequence end, running max per head
+    float mx[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) mx[n][0] = mx[n][1] = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int tok = t * 16 + g + ((r & 2) ? 8 : 0);
+          const float v = tok < valid ? sc[t][n][r] * scale_log2 : -INFINITY;
+          sc[t][n][r] = v;
+          mx[n][r & 1] = fmaxf(mx[n][r & 1], v);
+        }
+    float alpha[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float v = mx[n][c];
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        const float mnew = fmaxf(m[n][c], v);
+        alpha[n][c] = exp2f(m[n][c] - mnew);
+        m[n][c] = mnew;
+      }
+    float ls[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) ls[n][0] = ls[n][1] = 0.f;
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float pv = exp2f(sc[t][n][r] - m[n][r & 1]);
+          sc[t][n][r] = pv;
+          ls[n][r & 1] += pv;
+        }
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) l[n][c] = l[n][c] * alpha[n][c] + ls[n][c];
+#pragma unroll
+    for (int a = 0; a < KT; ++a)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) o[a][n][r] *= alpha[n][r & 1];
+
+    // O^T[d][head] += sum_token V[token][d] P[head][token]
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const uint32_t h01 = Mma<T>::pack(sc[t][n][0], sc[t][n][1]);
+        const uint32_t h23 = Mma<T>::pack(sc[t][n][2], sc[t][n][3]);
+        const float2 f01 = Mma<T>::unpack(h01), f23 = Mma<T>::unpack(h23);
+        const uint32_t l01 = Mma<T>::pack(sc[t][n][0] - f01.x, sc[t][n][1] - f01.y);
+        const uint32_t l23 = Mma<T>::pack(sc[t][n][2] - f23.x, sc[t][n][3] - f23.y);
+        bh[n][0] = movmatrix_trans(h01);
+        bh[n][1] = movmatrix_trans(h23);
+        bl[n][0] = movmatrix_trans(l01);
+        bl[n][1] = movmatrix_trans(l23);
+      }
+      // tokens of this thread's V fragments: t0 (+1) in a0/a1, t0+8 (+1) in a2/a3
+      const int t0 = t * 16 + tig * 2;
+      const bool tail = (t * 16 + 16) > valid;
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (tail) {
+        mlo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
+        mhi = (t0 + 8 < valid ? 0x0000ffffu : 0u) | (t0 + 9 < valid ? 0xffff0000u : 0u);
+      }
+      const int vrow = t * 16 + (mi >> 1) * 8 + ri;
+#pragma unroll
+      for (int a = 0; a < KT; ++a) {
+        const int dim = a * 16 + (mi & 1) * 8;
+        uint32_t f[4];
+        ldmatrix_x4_trans(f, vb + swz<B>(dim >> 6, vrow, (dim & 63) >> 3));
+        f[0] &= mlo;
+        f[1] &= mlo;
+        f[2] &= mhi;
+        f[3] &= mhi;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          Mma<T>::run(o[a][n], f, bh[n][0], bh[n][1]);
+          Mma<T>::run(o[a][n], f, bl[n][0], bl[n][1]);
+        }
+      }
+    }
+  }
+
+  // Write the segment: normalised output, or a partial for the merge kernel.
+  __device__ __forceinline__ void finish(const DecodeParams &p, int s, int h, bool complete,
+                                         int slot, int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+    const int G = p.group;
+    float lt[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float v = l[n][c];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        lt[n][c] = v;
+      }
+    if (complete) {
+      float *dst = p.out + ((int64_t)s * p.num_q_heads + (int64_t)h * G) * D;
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int head = n * 8 + tig * 2 + c;
+          if (head < G) {
+            const float inv = lt[n][c] > 0.f ? 1.f / lt[n][c] : 0.f;
+#pragma unroll
+            for (int a = 0; a < KT; ++a) {
+              dst[head * D + a * 16 + g] = o[a][n][c] * inv;
+              dst[head * D + a * 16 + g + 8] = o[a][n][2 + c] * inv;
+            }
+          }
+        }
+    } else {
+      float *po = p.part_o + (int64_t)slot * G * D;
+      float *pm = p.part_ml + (int64_t)slot * G * 2;
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int head = n * 8 + tig * 2 + c;
+          if (head < G) {
+#pragma unroll
+            for (int a = 0; a < KT; ++a) {
+              po[head * D + a * 16 + g] = o[a][n][c];
+              po[head * D + a * 16 + g + 8] = o[a][n][2 + c];
+            }
+            if (g == 0) {
+              pm[head * 2 + 0] = m[n][c];
+              pm[head * 2 + 1] = lt[n][c];
+            }
+          }
+        }
+    }
+  }
+};
+
+// ============================================================================
+// G == 1: CUDA-core path.
+// ============================================================================
+template <typename T, int D, int B>
+struct ScalarPath {
+  static constexpr int CPH = D / 16;   // 16-byte chunks per half row
+  static constexpr int DPL = D / 32;   // head-dim columns per lane in P.V
+  float acc[DPL];
+  float m, l;
+  float qr[D / 2];
+
+  // Chunk (box, index in box) that a lane of the given half reads at step i.
+  // D = 128: each half is one box; the order is rotated by 4 for the second
+  // half so the two halves of a token never hit the same banks.
+  __device__ __forceinline__ static void chunk(int i, int half, int &box, int &c) {
+    if constexpr (D == 128) {
+      box = half;
+      c = (i + 4 * half) & 7;
+    } else {
+      box = 0;
+      c = half * 4 + i;
+    }
+  }
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+    m = -INFINITY;
+    l = 0.f;
+  }
+
+  __device__ __forceinline__ void load_q(const uint8_t *qs, int /*G*/, int lane) {
+    const int half = lane & 1;
+#pragma unroll
+    for (int i = 0; i < CPH; ++i) {
+      int box, c;
+      chunk(i, half, box, c);
+      const uint4 v = *reinterpret_cast<const uint4 *>(qs + (box * 64 + c * 8) * 2);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = Mma<T>::unpack(w[e]);
+        qr[i * 8 + 2 * e] = f.x;
+        qr[i * 8 + 2 * e + 1] = f.y;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void tile(const uint8_t *ks, const uint8_t *vs, int valid,
+                                       float scale_log2, int lane) {
+    const int tk = lane >> 1, half = lane & 1;
+    constexpr int RR = B / 16;
+    float sr[RR];
+#pragma unroll
+    for (int rr = 0; rr < RR; ++rr) {
+      const int tok = rr * 16 + tk;
+      float dot = 0.f;
+#pragma unroll
+      for (int i = 0; i < CPH; ++i) {
+        int box, c;
+        chunk(i, half, box, c);
+        const uint4 v = *reinterpret_cast<const uint4 *>(ks + swz<B>(box, tok, c));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = Mma<T>::unpack(w[e]);
+          dot = fmaf(qr[i * 8 + 2 * e], f.x, dot);
+          dot = fmaf(qr[i * 8 + 2 * e + 1], f.y, dot);
+        }
+      }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      sr[rr] = tok < valid ? dot * scale_log2 : -INFINITY;
+    }
+    float mx = sr[0];
+#pragma unroll
+    for (int rr = 1; rr < RR; ++rr) mx = fmaxf(mx, sr[rr]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float mnew = fmaxf(m, mx);
+    const float alpha = exp2f(m - mnew);
+    m = mnew;
+    float ps = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < RR; ++rr) {
+      sr[rr] = exp2f(sr[rr] - mnew);
+      ps += sr[rr];
+    }
+    l = l * alpha + (half == 0 ? ps : 0.f);
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] *= alpha;
+
+#pragma unroll
+    for (int rr = 0; rr < RR; ++rr) {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const int tok = rr * 16 + t;
+        const float pt = __shfl_sync(0xffffffffu, sr[rr], 2 * t);
+        if (tok < valid) {   // warp-uniform: never touch V past the end
+          if constexpr (D == 128) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(
+                vs + swz<B>(lane >> 4, tok, (lane & 15) >> 1) + (lane & 1) * 8);
+            const float2 a = Mma<T>::unpack(v.x), b = Mma<T>::unpack(v.y);
+            acc[0] = fmaf(pt, a.x, acc[0]);
+            acc[1] = fmaf(pt, a.y, acc[1]);
+            acc[2] = fmaf(pt, b.x, acc[2]);
+            acc[3] = fmaf(pt, b.y, acc[3]);
+          } else {
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(
+                vs + swz<B>(0, tok, lane >> 2) + (lane & 3) * 4);
+            const float2 a = Mma<T>::unpack(v);
+            acc[0] = fmaf(pt, a.x, acc[0]);
+            acc[1] = fmaf(pt, a.y, acc[1]);
+          }
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void finish(const DecodeParams &p, int s, int h, bool complete,
+                                         int slot, int lane) {
+    float lt = l;
+#pragma unroll
+    for (int x = 1; x < 32; x <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, x);
+    if (complete) {
+      float *dst = p.out + ((int64_t)s * p.num_q_heads + h) * D + lane * DPL;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      if constexpr (DPL == 4) {
+        *reinterpret_cast<float4 *>(dst) =
+            make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      } else {
+        *reinterpret_cast<float2 *>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+      }
+    } else {
+      float *po = p.part_o + (int64_t)slot * D + lane * DPL;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) po[k] = acc[k];
+      if (lane == 0) {
+        p.part_ml[(int64_t)slot * 2 + 0] = m;
+        p.part_ml[(int64_t)slot * 2 + 1] = lt;
+      }
+    }
+  }
+};
+
+// ============================================================================
+// The attention kernel.
+// ============================================================================
+
+// Lane-parallel description of up to 32 consecutive tiles of one sequence.
+struct TileBatch {
+  int s, L, nb;      // warp-uniform
+  int n;             // number of tiles in the batch (0 = none)
+  int my_h, my_j, my_id;   // this lane's tile
+};
+
+template <int B>
+__device__ __forceinline__ void make_batch(const DecodeParams &p, TileBatch &tb, int s, int L,
+                                           int nb, int h, int j, int64_t remaining, int lane) {
+  tb.s = s;
+  tb.L = L;
+  tb.nb = nb;
+  const int64_t left_in_seq = (int64_t)p.num_kv_heads * nb - ((int64_t)h * nb + j);
+  int64_t n = left_in_seq < remaining ? left_in_seq : remaining;
+  tb.n = n < 32 ? (int)n : 32;
+  tb.my_h = 0;
+  tb.my_j = 0;
+  tb.my_id = -1;
+  if (lane < tb.n) {
+    const int pos = h * nb + j + lane;
+    tb.my_h = pos / nb;
+    tb.my_j = pos - tb.my_h * nb;
+    tb.my_id = __ldg(p.block_tables + (int64_t)s * p.max_blocks + tb.my_j);
+  }
+}
+
+template <typename T, int D, int B, int NT, int NW>
+__global__ void __launch_bounds__(NW * 32)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+  constexpr int TILE = B * D * 2;
+  constexpr int STAGE = 2 * TILE;
+  const int G = p.group;
+  const int qbytes = G * D * 2;
+  const int nstage = p.nstage;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.num_seqs, Hkv = p.num_kv_heads;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // per-warp regions
+  uint8_t *stages = smem + (size_t)warp * nstage * STAGE;
+  uint8_t *qslots = smem + (size_t)NW * nstage * STAGE + (size_t)warp * nstage * qbytes;
+  TileInfo *info = reinterpret_cast<TileInfo *>(smem + (size_t)NW * nstage * (STAGE + qbytes)) +
+                   warp * nstage;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(
+                       smem + (size_t)NW * nstage * (STAGE + qbytes + sizeof(TileInfo))) +
+                   warp * nstage;
+
+  __shared__ long long red[NW];
+  __shared__ int loc_s[NW];
+  __shared__ long long loc_base[NW];
+
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  if (lane == 0)
+    for (int k = 0; k < nstage; ++k) mbar_init(&bars[k], 1);
+
+  // ---- plan: total tiles, this CTA's warp ranges ---------------------------
+  long long mine = 0;
+  for (int s = threadIdx.x; s < S; s += NW * 32) {
+    const int nb = seq_blocks<B>(p, s, blockIdx.x == 0);
+    mine += nb;
+    if (nb == 0 && (s % gridDim.x) == blockIdx.x) {   // empty sequence: zero rows
+      float4 *row = reinterpret_cast<float4 *>(p.out + (int64_t)s * p.num_q_heads * D);
+      for (int k = 0; k < p.num_q_heads * D / 4; ++k) row[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, x);
+  if (lane == 0) red[warp] = mine;
+  __syncthreads();
+  long long tot = 0;
+#pragma unroll
+  for (int k = 0; k < NW; ++k) tot += red[k];
+  const long long U = tot * Hkv;
+  const long long w_total = (long long)gridDim.x * NW;
+  long long w_active = 0;
+  if (U > 0) {
+    w_active = (U + p.min_tiles - 1) / p.min_tiles;
+    if (w_active > w_total) w_active = w_total;
+  }
+  const long long w = (long long)blockIdx.x * NW + warp;
+  const bool active = w < w_active;
+  const long long u0 = active ? (w * U) / w_active : 0;
+  const long long u1 = active ? ((w + 1) * U) / w_active : 0;
+
+  // Locate the sequence holding each active warp's first tile: a chunked
+  // block-wide prefix sum over the per-sequence block counts.
+  long long cta_max_u0 = -1;
+  for (int k = 0; k < NW; ++k) {
+    const long long wk = (long long)blockIdx.x * NW + k;
+    if (wk < w_active) cta_max_u0 = (wk * U) / w_active;
+  }
+  if (cta_max_u0 >= 0) {
+    long long run = 0;
+    for (int c0 = 0; c0 < S; c0 += NW * 32) {
+      const int s = c0 + threadIdx.x;
+      const int nb = s < S ? seq_blocks<B>(p, s, false) : 0;
+      int incl = nb;
+#pragma unroll
+      for (int x = 1; x < 32; x <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, x);
+        if (lane >= x) incl += v;
+      }
+      __syncthreads();
+      if (lane == 31) red[warp] = incl;
+      __syncthreads();
+      long long before_warp = 0, chunk_tot = 0;
+#pragma unroll
+      for (int k = 0; k < NW; ++k) {
+        if (k < warp) before_warp += red[k];
+        chunk_tot += red[k];
+      }
+      const long long before = run + before_warp + incl - nb;   // blocks before seq s
+      if (nb > 0) {
+        const long long lo = before * Hkv, hi = (before + nb) * Hkv;
+        for (int k = 0; k < NW; ++k) {
+          const long long wk = (long long)blockIdx.x * NW + k;
+          if (wk < w_active) {
+            const long long uk = (wk * U) / w_active;
+            if (uk >= lo && uk < hi) {
+              loc_s[k] = s;
+              loc_base[k] = lo;
+            }
+          }
+        }
+      }
+      run += chunk_tot;
+      if (run * Hkv > cta_max_u0) break;
+    }
+  }
+  __syncthreads();
+  if (lane == 0) fence_barrier_init();
+  __syncwarp();
+
+  int64_t *meta = p.meta + w * kMetaWords;
+  if (!active) {
+    if (lane == 0) {
+      meta[0] = 0; meta[1] = 0; meta[2] = 0; meta[3] = U;
+      meta[4] = w_active; meta[5] = 0; meta[6] = 0; meta[7] = 0;
+    }
+    return;
+  }
+
+  // ---- this warp's first tile -----------------------------------------------
+  const int s0 = loc_s[warp];
+  const long long base0 = loc_base[warp];
+  const int L0 = seq_len_clamped<B>(p, s0);
+  const int nb0 = ceil_div_i(L0, B);
+  const long long r0 = u0 - base0;
+  const int h0 = (int)(r0 / nb0);
+  const int j0 = (int)(r0 - (long long)h0 * nb0);
+  if (lane == 0) {
+    const long long seg_lo = base0 + (long long)h0 * nb0;
+    meta[0] = u0; meta[1] = seg_lo; meta[2] = seg_lo + nb0; meta[3] = U;
+    meta[4] = w_active; meta[5] = s0; meta[6] = h0; meta[7] = 1;
+  }
+  const long long ntiles = u1 - u0;
+
+  // ---- issue cursor ---------------------------------------------------------
+  TileBatch cur, nxt;
+  long long issued = 0;          // tiles issued so far
+  int cur_k = 0;                 // next tile of `cur` to issue
+  make_batch<B>(p, cur, s0, L0, nb0, h0, j0, ntiles, lane);
+  auto follow = [&](const TileBatch &b, long long remaining_after) {
+    // the batch that comes after b in the walk
+    TileBatch r;
+    r.n = 0;
+    r.s = b.s; r.L = b.L; r.nb = b.nb; r.my_h = 0; r.my_j = 0; r.my_id = -1;
+    if (remaining_after <= 0) return r;
+    const int last_h = __shfl_sync(0xffffffffu, b.my_h, b.n - 1);
+    const int last_j = __shfl_sync(0xffffffffu, b.my_j, b.n - 1);
+    int h = last_h, j = last_j + 1;
+    int s = b.s, L = b.L, nb = b.nb;
+    if (j == nb) { j = 0; ++h; }
+    while (h >= Hkv || nb == 0) {   // next sequence with tiles
+      ++s;
+      if (s >= S) return r;
+      L = seq_len_clamped<B>(p, s);
+      nb = ceil_div_i(L, B);
+      h = 0;
+      j = 0;
+    }
+    make_batch<B>(p, r, s, L, nb, h, j, remaining_after, lane);
+    return r;
+  };
+  nxt = follow(cur, ntiles - cur.n);
+
+  const uint8_t *qbase = p.q;
+  auto issue = [&](int stage) {
+    if (cur_k == cur.n) {
+      cur = nxt;
+      cur_k = 0;
+      nxt = follow(cur, ntiles - issued - cur.n);
+    }
+    const int h = __shfl_sync(0xffffffffu, cur.my_h, cur_k);
+    const int j = __shfl_sync(0xffffffffu, cur.my_j, cur_k);
+    const int id = __shfl_sync(0xffffffffu, cur.my_id, cur_k);
+    if (lane == 0) {
+      int flags = 0;
+      if (j == 0 || issued == 0) flags |= TF_FIRST;
+      if (j == cur.nb - 1 || issued == ntiles - 1) flags |= TF_LAST;
+      if (j == 0) flags |= TF_J0;
+      if (j == cur.nb - 1) flags |= TF_JEND;
+      const bool ok = id >= 0 && id < p.num_blocks;
+      if (!ok) {
+        flags |= TF_SKIP;
+        flag_error(PA_DEVERR_BLOCK_ID);
+      }
+      const int valid = min(B, cur.L - j * B);
+      TileInfo ti;
+      ti.s = cur.s; ti.h = h; ti.j = j; ti.valid = valid; ti.flags = flags;
+      ti.pad0 = ti.pad1 = ti.pad2 = 0;
+      info[stage] = ti;
+      const uint32_t bytes = (ok ? STAGE : 0) + ((flags & TF_FIRST) ? qbytes : 0);
+      uint64_t *bar = &bars[stage];
+      if (bytes) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, bytes);
+        if (ok) {
+          const int row = (id * Hkv + h) * B;
+          uint8_t *kd = stages + (size_t)stage * STAGE;
+#pragma unroll
+          for (int bx = 0; bx < D / 64; ++bx) {
+            tma_load_2d(kd + bx * (B * 128), &kmap, bx * 64, row, bar);
+            tma_load_2d(kd + TILE + bx * (B * 128), &vmap, bx * 64, row, bar);
+          }
+        }
+        if (flags & TF_FIRST)
+          bulk_load(qslots + (size_t)stage * qbytes,
+                    qbase + ((int64_t)cur.s * p.num_q_heads + (int64_t)h * G) * (D * 2), qbytes,
+                    bar);
+      } else {
+        mbar_arrive(bar);
+      }
+    }
+    ++cur_k;
+    ++issued;
+  };
+
+  const int pre = ntiles < nstage ? (int)ntiles : nstage;
+  for (int k = 0; k < pre; ++k) issue(k);
+
+  // ---- consume --------------------------------------------------------------
+  using Path = typename std::conditional<NT == 0, ScalarPath<T, D, B>, MmaPath<T, D, B, (NT > 0 ? NT : 1)>>::type;
+  Path st;
+  st.reset();
+  bool seg_from0 = false;
+  int seg_index = 0;
+  for (long long i = 0; i < ntiles; ++i) {
+    const int stage = (int)(i % nstage);
+    const uint32_t parity = (uint32_t)((i / nstage) & 1);
+    if (!mbar_wait_bounded(&bars[stage], parity, kWaitLimitNs)) {
+      if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+      // drain the copies still in flight, then leave
+      for (long long k = i + 1; k < i + nstage && k < issued; ++k)
+        mbar_wait_bounded(&bars[k % nstage], (uint32_t)((k / nstage) & 1), kDrainLimitNs);
+      return;
+    }
+    const TileInfo ti = info[stage];
+    if (ti.flags & TF_FIRST) {
+      st.reset();
+      st.load_q(qslots + (size_t)stage * qbytes, G, lane);
+      seg_from0 = (ti.flags & TF_J0) != 0;
+    }
+    if (!(ti.flags & TF_SKIP)) {
+      const uint8_t *ks = stages + (size_t)stage * STAGE;
+      if constexpr (NT == 0) {
+        st.tile(ks, ks + TILE, ti.valid, p.scale_log2, lane);
+      } else {
+        st.tile(smem_addr(ks), smem_addr(ks + TILE), ti.valid, p.scale_log2, lane);
+      }
+    }
+    if (ti.flags & TF_LAST) {
+      const bool complete = seg_from0 && (ti.flags & TF_JEND);
+      st.finish(p, ti.s, ti.h, complete, (int)(2 * w + (seg_index == 0 ? 0 : 1)), lane);
+      ++seg_index;
+    }
+    __syncwarp();
+    if (i + nstage < ntiles) issue(stage);
+  }
+}
+
+// ============================================================================
+// Merge of split segments.  Block b looks at the boundary between warps b-1
+// and b; it merges the segment that boundary cuts if it is the first
+// boundary inside that segment.
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(128)
+    paged_decode_merge_kernel(float *out, const int64_t *meta, const float *part_ml,
+                              const float *part_o, int num_q_heads, int group) {
+  const long long b = (long long)blockIdx.x + 1;
+  const int64_t *mb = meta + b * kMetaWords;
+  if (mb[7] == 0) return;
+  const long long u0b = mb[0], lo = mb[1], hi = mb[2], U = mb[3], wa = mb[4];
+  if (lo >= u0b) return;                  // segment starts at this boundary
+  const long long u0a = meta[(b - 1) * kMetaWords + 0];
+  if (lo < u0a) return;                   // an earlier boundary cuts it first
+  const int s = (int)mb[5], h = (int)mb[6];
+  const int G = group;
+  const long long first_slot = 2 * (b - 1) + (lo == u0a ? 0 : 1);
+  long long last_w = b;
+  while (last_w + 1 < wa && ((last_w + 1) * U) / wa < hi) ++last_w;
+  const long long n = 1 + (last_w - b + 1);
+  float *dst = out + ((int64_t)s * num_q_heads + (int64_t)h * G) * D;
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int head = idx / D;
+    float M = -INFINITY;
+    for (long long k = 0; k < n; ++k) {
+      const long long slot = k == 0 ? first_slot : 2 * (b + k - 1);
+      M = fmaxf(M, part_ml[(slot * G + head) * 2]);
+    }
+    float num = 0.f, den = 0.f;
+    for (long long k = 0; k < n; ++k) {
+      const long long slot = k == 0 ? first_slot : 2 * (b + k - 1);
+      const float mk = part_ml[(slot * G + head) * 2];
+      const float wgt = mk == -INFINITY ? 0.f : exp2f(mk - M);
+      num = fmaf(wgt, part_o[slot * G * D + idx], num);
+      den = fmaf(wgt, part_ml[(slot * G + head) * 2 + 1], den);
+    }
+    dst[idx] = den > 0.f ? num / den : 0.f;
+  }
+}
+
+}  // namespace pa

@@ -19,3 +19,14 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("test marked gpu but no CUDA device is visible")
     return torch.device("cuda", 0)
+
+
+@pytest.fixture(scope="session")
+def pa():
+    """The binding, with libpa.so built in-tree first (nvcc cross-compiles
+    for sm_100a without a GPU)."""
+    from paged_kv_cache_414_b200 import build
+    build.build()
+    import paged_kv_cache_414_b200 as mod
+    mod.lib()
+    return mod
