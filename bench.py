@@ -166,6 +166,22 @@ def cpu_cores_used() -> int:
         return os.cpu_count() or 1
 
 
+def rank_reduce(x: float, op: str, world: int, device=None) -> float:
+    """Max or sum of a scalar over all ranks (identity on one rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_seed(name: str, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return W.SEEDS[name] + 1000 * rank
+
+
 # ----------------------------------------------------------------------------- workload
 
 class Workload:
@@ -176,13 +192,14 @@ class Workload:
         self.name = name
         sh = W.SHAPES[name]
         self.shape = sh
-        rng = np.random.default_rng(W.SEEDS[name] + 1000 * seed_offset)
+        seed = rank_seed(name, seed_offset)
+        rng = np.random.default_rng(seed)
         lens = {"gqa8b": W.lens_gqa8b, "13b": W.lens_13b}.get(name, W.lens_long)(rng)
         B = sh.block_size
         grow = math.ceil(steps_total / B) + 1
         need = sum(math.ceil(int(L) / B) + grow for L in lens)
         maxb = max(math.ceil((int(L) + steps_total) / B) for L in lens)
-        self.batch = W.make_decode_batch(sh, lens, W.SEEDS[name] + 1000 * seed_offset,
+        self.batch = W.make_decode_batch(sh, lens, seed,
                                          device=device, num_blocks=int(need * 1.1),
                                          max_blocks_per_seq=maxb, rng=rng)
         self.lens0 = lens.astype(np.int64)
@@ -283,19 +300,8 @@ def run_b200(args, rank, world, local_rank):
     bytes_steps = [wl.bytes_per_step(Wm + k) for k in range(K)]
     my_bytes = float(sum(bytes_steps))
 
-    def reduce_max(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def reduce_sum(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+    reduce_max = lambda x: rank_reduce(x, "max", world, dev)   # noqa: E731
+    reduce_sum = lambda x: rank_reduce(x, "sum", world, dev)   # noqa: E731
 
     ms_max = reduce_max(ms_total)
     all_bytes = reduce_sum(my_bytes)
@@ -482,20 +488,23 @@ def oracle_step_sample(wl, step: int, seqs):
 
 
 def cpu_baseline(wl, seconds: float):
+    """The oracle on a bounded sample of the workload: whole steps of random
+    sequences until about `seconds` of CPU work are spent."""
     rng = np.random.default_rng(0)
-    order = rng.permutation(wl.S)
-    spent, nbytes, done = 0.0, 0, []
-    for s in order:
-        dt, nb = oracle_step_sample(wl, 0, [int(s)])
-        spent += dt
-        nbytes += nb
-        done.append(int(s))
-        if spent >= seconds:
-            break
+    spent, nbytes, done, step = 0.0, 0, 0, 0
+    while spent < seconds and step < 64:
+        for s in rng.permutation(wl.S):
+            dt, nb = oracle_step_sample(wl, step, [int(s)])
+            spent += dt
+            nbytes += nb
+            done += 1
+            if spent >= seconds:
+                break
+        step += 1
     return {"value": round(nbytes / spent / 1e9, 4), "unit": "GB/s", "cores": cpu_cores_used(),
             "kind": "oracle",
-            "sample": f"{len(done)} of {wl.S} sequences of one step of the same workload "
-                      f"(oracle cache write + fp64 attention), {spent:.1f} s of CPU work"}
+            "sample": f"{done} sequence-steps of the same workload ({wl.S} sequences per step; "
+                      f"oracle cache write + fp64 attention), {spent:.1f} s of CPU work"}
 
 
 def run_reference(args, rank, world):
