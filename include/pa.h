@@ -142,6 +142,37 @@ int pa_paged_decode_attention(float *out, const void *q, const void *k_cache,
                               pa_stream_t stream);
 
 /*
+ * Allocation-free variant of pa_paged_decode_attention (no counterpart in the
+ * pages: an integration convenience).  Same arguments, same result, but no
+ * workspace argument: the split-context scratch lives in a fixed array of
+ * PA_NO_ALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library keeps until the process exits.  It is meant for callers
+ * that cannot allocate device memory themselves -- a plugin that only gets
+ * input and output buffers from a host framework owning all device memory,
+ * or a latency-critical caller where cudaMalloc (which may synchronise the
+ * device, or fail under memory pressure) is not allowed.  The call itself
+ * makes no device allocation and frees nothing.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call on a device shares the one array, which keeps the
+ * last call's contents (nothing in it needs clearing between calls): calls
+ * that may overlap on the GPU -- on different streams, or from different
+ * threads -- race and must be serialised by the caller.  Returns
+ * PA_ERR_WORKSPACE when the launch would need more than
+ * PA_NO_ALLOC_SCRATCH_BYTES (pa_paged_decode_workspace_bytes tells the need);
+ * otherwise as pa_paged_decode_attention.
+ */
+#define PA_NO_ALLOC_SCRATCH_BYTES (16u << 20)
+int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       const int32_t *context_lens, float scale,
+                                       int num_kv_heads, int num_seqs, int num_q_heads,
+                                       int head_dim, int block_size, int max_blocks_per_seq,
+                                       int max_context_len, int num_blocks, pa_dtype dtype,
+                                       pa_stream_t stream);
+
+/*
  * Override the decode launch heuristics for this process (0 = automatic):
  * stages of the per-warp copy ring, CTAs per SM, and the fewest tiles
  * ((sequence, kv head, block) units) a warp is given.  Affects calls made

@@ -68,6 +68,8 @@ def _declare(L):
         "pa_paged_decode_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
         "pa_paged_decode_attention": (i32, [vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                             i32, i32, i32, i32, vp, sz, vp]),
+        "pa_paged_decode_attention_no_alloc": (i32, [vp, vp, vp, vp, vp, vp, f32, i32, i32, i32,
+                                                     i32, i32, i32, i32, i32, i32, vp]),
         "pa_decode_tuning": (i32, [i32, i32, i32]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
         "pa_device_error": (i32, [c.POINTER(c.c_uint), i32]),
@@ -194,6 +196,33 @@ def pa_paged_decode_attention(out, q, k_cache, v_cache, block_tables, context_le
         int(max_context_len), NB, _dtype_code(k_cache), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_paged_decode_attention")
+    return out
+
+
+def pa_paged_decode_attention_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens,
+                                       scale, num_kv_heads, max_context_len=None, stream=None):
+    """pa_paged_decode_attention without a workspace: the library's own fixed
+    scratch array is used, and nothing is allocated (not even here), for
+    callers that cannot allocate device memory.  Calls that may overlap on
+    the GPU share that scratch and must be serialised by the caller."""
+    torch = _torch()
+    S, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    if Hkv != num_kv_heads or D2 != D:
+        raise ValueError("q / cache shapes disagree")
+    if tuple(out.shape) != (S, Hq, D):
+        raise ValueError("out must be [num_seqs, num_q_heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables [S, max_blocks] / context_lens [S] expected")
+    maxb = int(block_tables.shape[1])
+    if max_context_len is None:
+        max_context_len = maxb * B
+    st = lib().pa_paged_decode_attention_no_alloc(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), float(scale), Hkv, S, Hq, D, B, maxb,
+        int(max_context_len), NB, _dtype_code(k_cache), _stream(stream))
+    _check(st, "pa_paged_decode_attention_no_alloc")
     return out
 
 

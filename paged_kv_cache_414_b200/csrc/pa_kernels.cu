@@ -215,6 +215,36 @@ int current_device(int *dev) { return cudaGetDevice(dev) == cudaSuccess ? PA_OK 
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for pa_paged_decode_attention_no_alloc: a fixed array in device
+// global memory, part of the library's module, so that entry point needs no
+// allocation.  Every GPU that loads the library holds these bytes until the
+// process exits.  In host code the name is only a stand-in for the device
+// array: its device address comes from cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // PA_NO_ALLOC_SCRATCH_BYTES
+static __device__ __align__(256) unsigned char g_no_alloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_no_alloc_scratch on the current device `dev`, looked up
+// on the first call for that device (which must therefore not be inside a
+// stream capture) and cached.
+int no_alloc_scratch(int dev, void **out) {
+  static std::mutex mu;
+  static void *ptrs[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr)
+      return PA_ERR_CUDA;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *pa_status_string(int status) {
@@ -337,6 +367,46 @@ int pa_device_error(unsigned *flags, int clear) {
   }
   if (flags) *flags = v;
   return v ? PA_ERR_DEVICE_BOUNDS : PA_OK;
+}
+
+int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       const int32_t *context_lens, float scale,
+                                       int num_kv_heads, int num_seqs, int num_q_heads,
+                                       int head_dim, int block_size, int max_blocks_per_seq,
+                                       int max_context_len, int num_blocks, pa_dtype dtype,
+                                       pa_stream_t stream) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || head_dim <= 0 || block_size <= 0)
+    return PA_ERR_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_ARG;
+  if (!supported_shape(head_dim, block_size) || num_q_heads / num_kv_heads > 16)
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
+      (long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_ARG;
+  if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PA_ERR_ARG;
+  int dev;
+  if (current_device(&dev) != PA_OK || dev >= kMaxDevices) return PA_ERR_CUDA;
+  const int sms = sm_count(dev);
+  if (sms <= 0) return PA_ERR_CUDA;
+  void *scratch = nullptr;
+  const int st = no_alloc_scratch(dev, &scratch);
+  if (st != PA_OK) return st;
+  // The scratch needs no clearing: every descriptor and partial the merge
+  // reads is written by the same call first.  A launch that needs more than
+  // kNoAllocScratchBytes is refused by launch_decode with PA_ERR_WORKSPACE.
+  DecodeArgs a{out,         q,          k_cache,      v_cache,      block_tables,
+               context_lens, scale,     num_kv_heads, num_seqs,     num_q_heads,
+               head_dim,    block_size, max_blocks_per_seq, num_blocks, scratch,
+               kNoAllocScratchBytes, (cudaStream_t)stream};
+  if (dtype == PA_BF16) return dispatch_shape<__nv_bfloat16>(a, dev, sms);
+  return dispatch_shape<__half>(a, dev, sms);
 }
 
 int pa_decode_tuning(int nstage, int ctas_per_sm, int min_tiles_per_warp) {
