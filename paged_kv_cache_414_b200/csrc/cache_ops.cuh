@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256)
                              const int64_t *__restrict__ slot_mapping, long long num_vec,
                              int vec_per_row, int num_kv_heads, int block_size,
                              long long num_slots) {
+  allow_dependent_launch();   // the decode kernel may get scheduled meanwhile
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < num_vec; i += stride) {
     const long long row = i / vec_per_row;          // token * Hkv + head
@@ -50,6 +51,7 @@ __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                        const int64_t *__restrict__ block_mapping, long long vec_per_block,
                        int per_block, int num_blocks) {
+  allow_dependent_launch();
   const long long pair = blockIdx.y;
   const int64_t src = __ldg(block_mapping + 2 * pair);
   const int64_t dst = __ldg(block_mapping + 2 * pair + 1);

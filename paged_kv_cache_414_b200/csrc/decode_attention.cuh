@@ -15,8 +15,10 @@
 // the same number of bytes whatever the length mix.  A warp keeps one online
 // softmax state per segment; a segment that lies wholly inside one warp's
 // range is written to `out` directly, a segment cut by range boundaries
-// leaves one (max, sum, accumulator) partial per warp that touched it and a
-// second kernel merges them (split context).
+// leaves one (max, sum, accumulator) partial per warp that touched it, and
+// the last of those warps to finish merges them (split context): each warp
+// takes a ticket from an atomic counter of the segment after publishing its
+// partial; nobody waits, so there is no second kernel and no spin.
 //
 // Data movement.  Each warp owns a ring of `nstage` shared-memory stages and
 // issues its own copies: one 2-D TMA box per 64 head-dim columns of the K
@@ -47,7 +49,7 @@ namespace pa {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a copy never takes this long
 constexpr uint64_t kDrainLimitNs = 20000000ull;    // 20 ms to drain after a time-out
-constexpr int kMetaWords = 8;                      // int64 words per warp descriptor
+constexpr int kTicketCountBits = 24;               // ticket word: epoch << 24 | count
 
 // Tile flags.
 enum : int {
@@ -59,7 +61,8 @@ enum : int {
 };
 
 struct TileInfo {
-  int s, h, j, valid, flags, pad0, pad1, pad2;
+  int s, h, j, valid, flags, nb;
+  long long u;   // global tile index
 };
 
 struct DecodeParams {
@@ -67,7 +70,8 @@ struct DecodeParams {
   const uint8_t *q;
   const int32_t *block_tables;
   const int32_t *context_lens;
-  int64_t *meta;       // [w_total][kMetaWords]
+  unsigned long long *tickets;   // [w_total]: epoch << 24 | arrivals, per split segment
+  unsigned long long epoch;      // unique per call, < 2^40, never 0
   float *part_ml;      // [2 * w_total][G][2]   (max in log2 units, sum)
   float *part_o;       // [2 * w_total][G][D]
   float scale_log2;    // scale * log2(e)
@@ -275,7 +279,7 @@ struct MmaPath {
     }
   }
 
-  // Write the segment: normalised output, or a partial for the merge kernel.
+  // Write the segment: normalised output, or a partial for the merge.
   __device__ __forceinline__ void finish(const DecodeParams &p, int s, int h, bool complete,
                                          int slot, int lane) {
     const int g = lane >> 2, tig = lane & 3;
@@ -478,6 +482,142 @@ struct ScalarPath {
 };
 
 // ============================================================================
+// Split-context merge, done by the last warp to finish a split segment.
+// ============================================================================
+
+// First tile of warp c when U tiles are cut into wa equal ranges, and the
+// warp whose range holds tile u.
+__device__ __forceinline__ long long warp_start(long long c, long long U, long long wa) {
+  return c * U / wa;
+}
+__device__ __forceinline__ long long warp_of(long long u, long long U, long long wa) {
+  return ((u + 1) * wa - 1) / U;
+}
+
+// Arrival number (0-based) at a split segment's counter for this call.  The
+// counter word holds the call's epoch in its high bits, so a word left by an
+// earlier call (or zero-filled memory) reads as no arrival yet.
+__device__ __forceinline__ unsigned take_ticket(unsigned long long *t, unsigned long long epoch) {
+  unsigned long long cur = atomicAdd(t, 0ull);
+  const unsigned long long mask = (1ull << kTicketCountBits) - 1;
+  for (int it = 0; it < (1 << 20); ++it) {
+    const unsigned cnt = ((cur >> kTicketCountBits) == epoch) ? (unsigned)(cur & mask) : 0u;
+    const unsigned long long want = (epoch << kTicketCountBits) | (unsigned long long)(cnt + 1);
+    const unsigned long long prev = atomicCAS(t, cur, want);
+    if (prev == cur) return cnt;
+    cur = prev;
+  }
+  flag_error(PA_DEVERR_TIMEOUT);
+  return 0xffffffffu;
+}
+
+// Called by every warp right after it wrote its partial of the split segment
+// (s, h) = tiles [lo, hi).  The warp that arrives last merges all partials:
+// with M = max_i m_i, out = sum_i 2^(m_i - M) acc_i / sum_i 2^(m_i - M) l_i.
+template <int D, int GMAX>
+__device__ void merge_if_last(const DecodeParams &p, int s, int h, long long lo, long long hi,
+                              long long U, long long wa, int lane) {
+  constexpr int VPL = D / 32;
+  __threadfence();
+  __syncwarp();
+  const long long c_lo = warp_of(lo, U, wa), c_hi = warp_of(hi - 1, U, wa);
+  const long long n = c_hi - c_lo + 1;
+  unsigned ticket = 0;
+  if (lane == 0) ticket = take_ticket(p.tickets + c_lo, p.epoch);
+  ticket = __shfl_sync(0xffffffffu, ticket, 0);
+  if ((long long)ticket != n - 1) return;
+  __threadfence();
+
+  const int G = p.group;
+  float *dst = p.out + ((int64_t)s * p.num_q_heads + (int64_t)h * G) * D + lane * VPL;
+  using VecT = typename std::conditional<VPL == 4, float4, float2>::type;
+  // Heads in chunks of GMAX.  Lane k reads partial k's (max, sum); the
+  // accumulators are read UNR partials at a time with every load issued
+  // before any is used, so the L2 latency is paid once per UNR partials.
+  constexpr int UNR = 4;
+  for (int g0 = 0; g0 < G; g0 += GMAX) {
+    float M[GMAX], den[GMAX], num[GMAX][VPL];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      M[g] = -INFINITY;
+      den[g] = 0.f;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) num[g][v] = 0.f;
+    }
+    for (long long k0 = 0; k0 < n; k0 += 32) {
+      const long long k = k0 + lane;
+      const bool ok = k < n;
+      const long long c = c_lo + k;
+      const long long slot = ok ? ((lo <= warp_start(c, U, wa)) ? 2 * c : 2 * c + 1) : 0;
+      const int cnt = (int)((n - k0) < 32 ? (n - k0) : 32);
+      float wk[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        const int head = g0 + g < G ? g0 + g : G - 1;
+        const float mk = ok ? __ldcg(p.part_ml + (slot * G + head) * 2) : -INFINITY;
+        const float lk = ok ? __ldcg(p.part_ml + (slot * G + head) * 2 + 1) : 0.f;
+        float cm = mk;
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, x));
+        const float Mn = fmaxf(M[g], cm);
+        const float so = Mn == -INFINITY ? 0.f : exp2f(M[g] - Mn);
+        wk[g] = (mk == -INFINITY) ? 0.f : exp2f(mk - Mn);
+        float dl = wk[g] * lk;
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, x);
+        den[g] = den[g] * so + dl;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) num[g][v] *= so;
+        M[g] = Mn;
+      }
+      for (int j0 = 0; j0 < cnt; j0 += UNR) {
+        VecT buf[UNR][GMAX];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+          const int j = j0 + u < cnt ? j0 + u : cnt - 1;
+          const long long sj = __shfl_sync(0xffffffffu, slot, j);
+#pragma unroll
+          for (int g = 0; g < GMAX; ++g) {
+            const int head = g0 + g < G ? g0 + g : G - 1;
+            buf[u][g] = __ldcg(reinterpret_cast<const VecT *>(p.part_o + (sj * G + head) * D +
+                                                              lane * VPL));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+          const int j = j0 + u;
+#pragma unroll
+          for (int g = 0; g < GMAX; ++g) {
+            float wj = __shfl_sync(0xffffffffu, wk[g], j < cnt ? j : 0);
+            wj = j < cnt ? wj : 0.f;
+            num[g][0] = fmaf(wj, buf[u][g].x, num[g][0]);
+            num[g][1] = fmaf(wj, buf[u][g].y, num[g][1]);
+            if constexpr (VPL == 4) {
+              num[g][2] = fmaf(wj, reinterpret_cast<const float4 &>(buf[u][g]).z, num[g][2]);
+              num[g][3] = fmaf(wj, reinterpret_cast<const float4 &>(buf[u][g]).w, num[g][3]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      const int head = g0 + g;
+      if (head < G) {
+        const float inv = den[g] > 0.f ? 1.f / den[g] : 0.f;
+        if constexpr (VPL == 4) {
+          *reinterpret_cast<float4 *>(dst + head * D) =
+              make_float4(num[g][0] * inv, num[g][1] * inv, num[g][2] * inv, num[g][3] * inv);
+        } else {
+          *reinterpret_cast<float2 *>(dst + head * D) =
+              make_float2(num[g][0] * inv, num[g][1] * inv);
+        }
+      }
+    }
+  }
+}
+
+// ============================================================================
 // The attention kernel.
 // ============================================================================
 
@@ -509,7 +649,7 @@ __device__ __forceinline__ void make_batch(const DecodeParams &p, TileBatch &tb,
 }
 
 template <typename T, int D, int B, int NT, int NW>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
   constexpr int TILE = B * D * 2;
@@ -542,6 +682,10 @@ __global__ void __launch_bounds__(NW * 32)
   }
   if (lane == 0)
     for (int k = 0; k < nstage; ++k) mbar_init(&bars[k], 1);
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: everything above overlaps its tail; nothing below may run before
+  // its writes (the step's new K/V, say) are visible.
+  grid_dependency_wait();
 
   // ---- plan: total tiles, this CTA's warp ranges ---------------------------
   long long mine = 0;
@@ -621,14 +765,7 @@ __global__ void __launch_bounds__(NW * 32)
   if (lane == 0) fence_barrier_init();
   __syncwarp();
 
-  int64_t *meta = p.meta + w * kMetaWords;
-  if (!active) {
-    if (lane == 0) {
-      meta[0] = 0; meta[1] = 0; meta[2] = 0; meta[3] = U;
-      meta[4] = w_active; meta[5] = 0; meta[6] = 0; meta[7] = 0;
-    }
-    return;
-  }
+  if (!active) return;
 
   // ---- this warp's first tile -----------------------------------------------
   const int s0 = loc_s[warp];
@@ -638,11 +775,6 @@ __global__ void __launch_bounds__(NW * 32)
   const long long r0 = u0 - base0;
   const int h0 = (int)(r0 / nb0);
   const int j0 = (int)(r0 - (long long)h0 * nb0);
-  if (lane == 0) {
-    const long long seg_lo = base0 + (long long)h0 * nb0;
-    meta[0] = u0; meta[1] = seg_lo; meta[2] = seg_lo + nb0; meta[3] = U;
-    meta[4] = w_active; meta[5] = s0; meta[6] = h0; meta[7] = 1;
-  }
   const long long ntiles = u1 - u0;
 
   // ---- issue cursor ---------------------------------------------------------
@@ -698,7 +830,8 @@ __global__ void __launch_bounds__(NW * 32)
       const int valid = min(B, cur.L - j * B);
       TileInfo ti;
       ti.s = cur.s; ti.h = h; ti.j = j; ti.valid = valid; ti.flags = flags;
-      ti.pad0 = ti.pad1 = ti.pad2 = 0;
+      ti.nb = cur.nb;
+      ti.u = u0 + issued;
       info[stage] = ti;
       const uint32_t bytes = (ok ? STAGE : 0) + ((flags & TF_FIRST) ? qbytes : 0);
       uint64_t *bar = &bars[stage];
@@ -762,52 +895,14 @@ __global__ void __launch_bounds__(NW * 32)
     if (ti.flags & TF_LAST) {
       const bool complete = seg_from0 && (ti.flags & TF_JEND);
       st.finish(p, ti.s, ti.h, complete, (int)(2 * w + (seg_index == 0 ? 0 : 1)), lane);
+      if (!complete) {
+        const long long lo = ti.u - ti.j;
+        merge_if_last<D, (NT == 0 ? 1 : 4)>(p, ti.s, ti.h, lo, lo + ti.nb, U, w_active, lane);
+      }
       ++seg_index;
     }
     __syncwarp();
     if (i + nstage < ntiles) issue(stage);
-  }
-}
-
-// ============================================================================
-// Merge of split segments.  Block b looks at the boundary between warps b-1
-// and b; it merges the segment that boundary cuts if it is the first
-// boundary inside that segment.
-// ============================================================================
-template <int D>
-__global__ void __launch_bounds__(128)
-    paged_decode_merge_kernel(float *out, const int64_t *meta, const float *part_ml,
-                              const float *part_o, int num_q_heads, int group) {
-  const long long b = (long long)blockIdx.x + 1;
-  const int64_t *mb = meta + b * kMetaWords;
-  if (mb[7] == 0) return;
-  const long long u0b = mb[0], lo = mb[1], hi = mb[2], U = mb[3], wa = mb[4];
-  if (lo >= u0b) return;                  // segment starts at this boundary
-  const long long u0a = meta[(b - 1) * kMetaWords + 0];
-  if (lo < u0a) return;                   // an earlier boundary cuts it first
-  const int s = (int)mb[5], h = (int)mb[6];
-  const int G = group;
-  const long long first_slot = 2 * (b - 1) + (lo == u0a ? 0 : 1);
-  long long last_w = b;
-  while (last_w + 1 < wa && ((last_w + 1) * U) / wa < hi) ++last_w;
-  const long long n = 1 + (last_w - b + 1);
-  float *dst = out + ((int64_t)s * num_q_heads + (int64_t)h * G) * D;
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int head = idx / D;
-    float M = -INFINITY;
-    for (long long k = 0; k < n; ++k) {
-      const long long slot = k == 0 ? first_slot : 2 * (b + k - 1);
-      M = fmaxf(M, part_ml[(slot * G + head) * 2]);
-    }
-    float num = 0.f, den = 0.f;
-    for (long long k = 0; k < n; ++k) {
-      const long long slot = k == 0 ? first_slot : 2 * (b + k - 1);
-      const float mk = part_ml[(slot * G + head) * 2];
-      const float wgt = mk == -INFINITY ? 0.f : exp2f(mk - M);
-      num = fmaf(wgt, part_o[slot * G * D + idx], num);
-      den = fmaf(wgt, part_ml[(slot * G + head) * 2 + 1], den);
-    }
-    dst[idx] = den > 0.f ? num / den : 0.f;
   }
 }
 

@@ -82,6 +82,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// ---------------------------------------------------------------- grid dependencies
+
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their writes are visible (returns at once without one).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next kernel on the stream be scheduled before this one finishes.
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 2-D tiled tensor copy global -> shared, completion counted in bytes on `bar`.

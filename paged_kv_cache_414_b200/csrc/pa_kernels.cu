@@ -59,6 +59,17 @@ std::atomic<int> g_tune_nstage{0};
 std::atomic<int> g_tune_ctas{0};
 std::atomic<int> g_tune_min_tiles{0};
 
+// Per-call epoch for the split-segment tickets: unique, non-zero, < 2^40.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> ctr{0};
+  const unsigned long long mask = (1ull << 40) - 1;
+  unsigned long long e;
+  do {
+    e = (ctr.fetch_add(1) + 1) & mask;
+  } while (e == 0);
+  return e;
+}
+
 struct DecodeLayout {
   int nstage, ctas_per_sm, grid, w_total, min_tiles;
   size_t smem;
@@ -75,7 +86,7 @@ size_t cta_smem(int D, int B, int G, int nstage) {
 }
 
 size_t workspace_for(int w_total, int G, int D, size_t *off_ml, size_t *off_o) {
-  size_t meta = round_up((size_t)w_total * pa::kMetaWords * sizeof(int64_t), 256);
+  size_t meta = round_up((size_t)w_total * sizeof(unsigned long long), 256);   // tickets
   size_t ml = round_up((size_t)2 * w_total * G * 2 * sizeof(float), 256);
   size_t o = round_up((size_t)2 * w_total * G * D * sizeof(float), 256);
   if (off_ml) *off_ml = meta;
@@ -83,29 +94,34 @@ size_t workspace_for(int w_total, int G, int D, size_t *off_ml, size_t *off_o) {
   return meta + ml + o;
 }
 
-// Stages per warp and CTAs per SM: as many stages as fit with two CTAs per SM
-// (at least three), else one CTA per SM.
-void choose_layout(int D, int B, int G, int sms, DecodeLayout *L) {
-  const size_t per_sm = 227 * 1024;   // usable shared memory per SM
+// CTAs per SM and stages per warp.  Each warp issues its own copies, so
+// resident warps are what keeps HBM busy; measured on B200, two stages per
+// warp with the most CTAs per SM beat deeper rings with fewer warps for every
+// workload shape (even one stage with twice the warps beat three stages).
+// So: the most CTAs per SM (at most 3) that registers and shared memory allow
+// with at least one stage, and up to two stages per warp.
+void choose_layout(int D, int B, int G, int sms, int regs_per_thread, DecodeLayout *L) {
+  const size_t per_sm = 228 * 1024;   // shared memory per SM
+  const size_t per_cta_reserved = 1024;
+  const size_t set = (size_t)kWarpsPerCta * stage_bytes(D, B, G);
   const int want_ctas = g_tune_ctas.load();
   const int want_stages = g_tune_nstage.load();
-  int ctas = 2, nst = 0;
-  for (int c : {2, 1}) {
-    const size_t budget = per_sm / c - 1024 - 256;
-    int n = (int)((budget - 1024) / ((size_t)kWarpsPerCta * stage_bytes(D, B, G)));
-    n = std::min(n, 8);
-    if (n >= 3 || c == 1) {
+  int reg_ctas = regs_per_thread > 0 ? 65536 / (regs_per_thread * kWarpsPerCta * 32) : 2;
+  reg_ctas = std::max(1, std::min(reg_ctas, 3));
+  auto stages_for = [&](int c) {
+    const size_t budget = per_sm / c - per_cta_reserved - 256;   // 256: static smem
+    return (int)((budget - 1024) / set);
+  };
+  int ctas = 1;
+  for (int c = reg_ctas; c >= 1; --c) {
+    if (stages_for(c) >= 1) {
       ctas = c;
-      nst = n;
       break;
     }
   }
-  if (want_ctas > 0) {
-    ctas = std::min(want_ctas, kMaxCtasPerSm);
-    const size_t budget = per_sm / ctas - 1024 - 256;
-    nst = (int)((budget - 1024) / ((size_t)kWarpsPerCta * stage_bytes(D, B, G)));
-  }
-  if (want_stages > 0) nst = std::min(nst, want_stages);
+  if (want_ctas > 0) ctas = std::min(want_ctas, kMaxCtasPerSm);
+  int nst = std::min(stages_for(ctas), 2);
+  if (want_stages > 0) nst = std::min(stages_for(ctas), want_stages);
   nst = std::max(nst, 1);
   L->nstage = nst;
   L->ctas_per_sm = ctas;
@@ -144,11 +160,19 @@ struct DecodeArgs {
 template <typename T, int D, int B, int NT>
 int launch_decode(const DecodeArgs &a, int dev, int sms) {
   const int G = a.num_q_heads / a.num_kv_heads;
+  auto kern = pa::paged_decode_kernel<T, D, B, NT, kWarpsPerCta>;
+  static std::atomic<int> regs_cache{0};
+  int regs = regs_cache.load();
+  if (regs == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PA_ERR_CUDA;
+    regs = fa.numRegs;
+    regs_cache.store(regs);
+  }
   DecodeLayout L;
-  choose_layout(D, B, G, sms, &L);
+  choose_layout(D, B, G, sms, regs, &L);
   if (a.workspace_bytes < L.workspace) return PA_ERR_WORKSPACE;
 
-  auto kern = pa::paged_decode_kernel<T, D, B, NT, kWarpsPerCta>;
   static std::atomic<size_t> attr_set[kMaxDevices];
   if (attr_set[dev].load() < L.smem) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem) !=
@@ -168,7 +192,8 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   p.q = static_cast<const uint8_t *>(a.q);
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
-  p.meta = reinterpret_cast<int64_t *>(ws + L.off_meta);
+  p.tickets = reinterpret_cast<unsigned long long *>(ws + L.off_meta);
+  p.epoch = next_epoch();
   p.part_ml = reinterpret_cast<float *>(ws + L.off_ml);
   p.part_o = reinterpret_cast<float *>(ws + L.off_o);
   p.scale_log2 = a.scale * 1.4426950408889634f;
@@ -181,12 +206,23 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   p.nstage = L.nstage;
   p.min_tiles = L.min_tiles;
 
-  kern<<<L.grid, kWarpsPerCta * 32, L.smem, a.stream>>>(kmap, vmap, p);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (L.w_total > 1) {
-    pa::paged_decode_merge_kernel<D><<<L.w_total - 1, 128, 0, a.stream>>>(
-        a.out, p.meta, p.part_ml, p.part_o, a.num_q_heads, G);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  // Programmatic dependent launch: the grid may be scheduled while the
+  // previous kernel on the stream (typically reshape_and_cache) is still
+  // running; the kernel waits for it (griddepcontrol.wait) before its first
+  // global-memory read.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(L.grid);
+  cfg.blockDim = dim3(kWarpsPerCta * 32);
+  cfg.dynamicSmemBytes = L.smem;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, kmap, vmap, p) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
   }
   return PA_OK;
 }
@@ -398,8 +434,9 @@ int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_
   void *scratch = nullptr;
   const int st = no_alloc_scratch(dev, &scratch);
   if (st != PA_OK) return st;
-  // The scratch needs no clearing: every descriptor and partial the merge
-  // reads is written by the same call first.  A launch that needs more than
+  // The scratch needs no clearing: every partial the merge reads is written
+  // by the same call first, and the split-segment counters carry the call's
+  // epoch, so counts left by an earlier call read as zero.  A launch that needs more than
   // kNoAllocScratchBytes is refused by launch_decode with PA_ERR_WORKSPACE.
   DecodeArgs a{out,         q,          k_cache,      v_cache,      block_tables,
                context_lens, scale,     num_kv_heads, num_seqs,     num_q_heads,
