@@ -15,10 +15,11 @@
 // the same number of bytes whatever the length mix.  A warp keeps one online
 // softmax state per segment; a segment that lies wholly inside one warp's
 // range is written to `out` directly, a segment cut by range boundaries
-// leaves one (max, sum, accumulator) partial per warp that touched it, and
-// the last of those warps to finish merges them (split context): each warp
-// takes a ticket from an atomic counter of the segment after publishing its
-// partial; nobody waits, so there is no second kernel and no spin.
+// leaves one (max, sum, accumulator) partial per warp that touched it
+// (split context).  A small merge kernel, launched as a programmatic
+// dependent so it starts as soon as the last streaming warp is done, combines
+// the partials: one warp per boundary between warp ranges.  The streaming
+// kernel itself never waits, fences or takes an atomic.
 //
 // Data movement.  Each warp owns a ring of `nstage` shared-memory stages and
 // issues its own copies: one 2-D TMA box per 64 head-dim columns of the K
@@ -49,7 +50,7 @@ namespace pa {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a copy never takes this long
 constexpr uint64_t kDrainLimitNs = 20000000ull;    // 20 ms to drain after a time-out
-constexpr int kTicketCountBits = 24;               // ticket word: epoch << 24 | count
+constexpr int kMetaWords = 8;                      // per-warp descriptor for the merge
 
 // Tile flags.
 enum : int {
@@ -70,8 +71,7 @@ struct DecodeParams {
   const uint8_t *q;
   const int32_t *block_tables;
   const int32_t *context_lens;
-  unsigned long long *tickets;   // [w_total]: epoch << 24 | arrivals, per split segment
-  unsigned long long epoch;      // unique per call, < 2^40, never 0
+  long long *meta;     // [w_total][kMetaWords]: each warp's range and first segment
   float *part_ml;      // [2 * w_total][G][2]   (max in log2 units, sum)
   float *part_o;       // [2 * w_total][G][D]
   float scale_log2;    // scale * log2(e)
@@ -494,40 +494,20 @@ __device__ __forceinline__ long long warp_of(long long u, long long U, long long
   return ((u + 1) * wa - 1) / U;
 }
 
-// Arrival number (0-based) at a split segment's counter for this call.  The
-// counter word holds the call's epoch in its high bits, so a word left by an
-// earlier call (or zero-filled memory) reads as no arrival yet.
-__device__ __forceinline__ unsigned take_ticket(unsigned long long *t, unsigned long long epoch) {
-  unsigned long long cur = atomicAdd(t, 0ull);
-  const unsigned long long mask = (1ull << kTicketCountBits) - 1;
-  for (int it = 0; it < (1 << 20); ++it) {
-    const unsigned cnt = ((cur >> kTicketCountBits) == epoch) ? (unsigned)(cur & mask) : 0u;
-    const unsigned long long want = (epoch << kTicketCountBits) | (unsigned long long)(cnt + 1);
-    const unsigned long long prev = atomicCAS(t, cur, want);
-    if (prev == cur) return cnt;
-    cur = prev;
-  }
-  flag_error(PA_DEVERR_TIMEOUT);
-  return 0xffffffffu;
+// Partial slot of part c (a warp) of the split segment that starts at tile lo.
+__device__ __forceinline__ long long part_slot(long long c, long long lo, long long U,
+                                               long long wa) {
+  return (lo <= warp_start(c, U, wa)) ? 2 * c : 2 * c + 1;
 }
 
-// Called by every warp right after it wrote its partial of the split segment
-// (s, h) = tiles [lo, hi).  The warp that arrives last merges all partials:
-// with M = max_i m_i, out = sum_i 2^(m_i - M) acc_i / sum_i 2^(m_i - M) l_i.
+// Merge all partials of the split segment (s, h) = tiles [lo, hi): with
+// M = max_i m_i, out = sum_i 2^(m_i - M) acc_i / sum_i 2^(m_i - M) l_i.
 template <int D, int GMAX>
-__device__ void merge_if_last(const DecodeParams &p, int s, int h, long long lo, long long hi,
-                              long long U, long long wa, int lane) {
+__device__ void merge_parts(const DecodeParams &p, int s, int h, long long lo, long long hi,
+                            long long U, long long wa, int lane) {
   constexpr int VPL = D / 32;
-  __threadfence();
-  __syncwarp();
   const long long c_lo = warp_of(lo, U, wa), c_hi = warp_of(hi - 1, U, wa);
   const long long n = c_hi - c_lo + 1;
-  unsigned ticket = 0;
-  if (lane == 0) ticket = take_ticket(p.tickets + c_lo, p.epoch);
-  ticket = __shfl_sync(0xffffffffu, ticket, 0);
-  if ((long long)ticket != n - 1) return;
-  __threadfence();
-
   const int G = p.group;
   float *dst = p.out + ((int64_t)s * p.num_q_heads + (int64_t)h * G) * D + lane * VPL;
   using VecT = typename std::conditional<VPL == 4, float4, float2>::type;
@@ -548,7 +528,7 @@ __device__ void merge_if_last(const DecodeParams &p, int s, int h, long long lo,
       const long long k = k0 + lane;
       const bool ok = k < n;
       const long long c = c_lo + k;
-      const long long slot = ok ? ((lo <= warp_start(c, U, wa)) ? 2 * c : 2 * c + 1) : 0;
+      const long long slot = ok ? part_slot(c, lo, U, wa) : 0;
       const int cnt = (int)((n - k0) < 32 ? (n - k0) : 32);
       float wk[GMAX];
 #pragma unroll
@@ -675,6 +655,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   __shared__ long long red[NW];
   __shared__ int loc_s[NW];
   __shared__ long long loc_base[NW];
+  __shared__ int loc_L[NW];
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&kmap);
@@ -686,95 +667,169 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   // stream: everything above overlaps its tail; nothing below may run before
   // its writes (the step's new K/V, say) are visible.
   grid_dependency_wait();
+  allow_dependent_launch();   // the split merge may be scheduled meanwhile
 
   // ---- plan: total tiles, this CTA's warp ranges ---------------------------
-  long long mine = 0;
-  for (int s = threadIdx.x; s < S; s += NW * 32) {
-    const int nb = seq_blocks<B>(p, s, blockIdx.x == 0);
-    mine += nb;
-    if (nb == 0 && (s % gridDim.x) == blockIdx.x) {   // empty sequence: zero rows
-      float4 *row = reinterpret_cast<float4 *>(p.out + (int64_t)s * p.num_q_heads * D);
-      for (int k = 0; k < p.num_q_heads * D / 4; ++k) row[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
-#pragma unroll
-  for (int x = 16; x > 0; x >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, x);
-  if (lane == 0) red[warp] = mine;
-  __syncthreads();
-  long long tot = 0;
-#pragma unroll
-  for (int k = 0; k < NW; ++k) tot += red[k];
-  const long long U = tot * Hkv;
+  // Every CTA reads all context lengths once, scans their block counts, and
+  // finds the sequence holding the first tile of each of its warps.
+  constexpr int NT_ = NW * 32;   // threads per CTA
+  constexpr int KMAX = 8;   // sequences per thread on the one-pass path
   const long long w_total = (long long)gridDim.x * NW;
-  long long w_active = 0;
-  if (U > 0) {
-    w_active = (U + p.min_tiles - 1) / p.min_tiles;
-    if (w_active > w_total) w_active = w_total;
-  }
   const long long w = (long long)blockIdx.x * NW + warp;
-  const bool active = w < w_active;
-  const long long u0 = active ? (w * U) / w_active : 0;
-  const long long u1 = active ? ((w + 1) * U) / w_active : 0;
-
-  // Locate the sequence holding each active warp's first tile: a chunked
-  // block-wide prefix sum over the per-sequence block counts.
-  long long cta_max_u0 = -1;
-  for (int k = 0; k < NW; ++k) {
+  long long U = 0, w_active = 0;
+  auto set_ranges = [&](long long tot) {
+    U = tot * Hkv;
+    w_active = 0;
+    if (U > 0) {
+      w_active = (U + p.min_tiles - 1) / p.min_tiles;
+      if (w_active > w_total) w_active = w_total;
+    }
+  };
+  auto warp_u0 = [&](int k) -> long long {   // first tile of this CTA's warp k, -1 if idle
     const long long wk = (long long)blockIdx.x * NW + k;
-    if (wk < w_active) cta_max_u0 = (wk * U) / w_active;
-  }
-  if (cta_max_u0 >= 0) {
-    long long run = 0;
-    for (int c0 = 0; c0 < S; c0 += NW * 32) {
-      const int s = c0 + threadIdx.x;
-      const int nb = s < S ? seq_blocks<B>(p, s, false) : 0;
-      int incl = nb;
+    return wk < w_active ? (wk * U) / w_active : -1;
+  };
+  auto zero_row = [&](int s) {   // empty sequence: zero output rows
+    float4 *row = reinterpret_cast<float4 *>(p.out + (int64_t)s * p.num_q_heads * D);
+    for (int k = 0; k < p.num_q_heads * D / 4; ++k) row[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  const int cap = p.max_blocks * B;
+  if (S <= NT_ * KMAX) {
+    // one pass: thread t owns sequences [t*K, t*K + K)
+    const int K = (S + NT_ - 1) / NT_;
+    const int sbeg = threadIdx.x * K;
+    int Lr[KMAX];
 #pragma unroll
-      for (int x = 1; x < 32; x <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, x);
-        if (lane >= x) incl += v;
-      }
-      __syncthreads();
-      if (lane == 31) red[warp] = incl;
-      __syncthreads();
-      long long before_warp = 0, chunk_tot = 0;
+    for (int k = 0; k < KMAX; ++k)
+      Lr[k] = (k < K && sbeg + k < S) ? __ldg(p.context_lens + sbeg + k) : 0;
+    int mine = 0;
 #pragma unroll
-      for (int k = 0; k < NW; ++k) {
-        if (k < warp) before_warp += red[k];
-        chunk_tot += red[k];
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < K && sbeg + k < S) {
+        int L = Lr[k];
+        if (L < 0 || L > cap) {
+          if (blockIdx.x == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
+          L = L < 0 ? 0 : cap;
+        }
+        Lr[k] = L;
+        mine += ceil_div_i(L, B);
+        if (L == 0 && ((sbeg + k) % gridDim.x) == blockIdx.x) zero_row(sbeg + k);
       }
-      const long long before = run + before_warp + incl - nb;   // blocks before seq s
-      if (nb > 0) {
-        const long long lo = before * Hkv, hi = (before + nb) * Hkv;
-        for (int k = 0; k < NW; ++k) {
-          const long long wk = (long long)blockIdx.x * NW + k;
-          if (wk < w_active) {
-            const long long uk = (wk * U) / w_active;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int x = 1; x < 32; x <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, x);
+      if (lane >= x) incl += v;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    long long before_warp = 0, tot = 0;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) {
+      if (k < warp) before_warp += red[k];
+      tot += red[k];
+    }
+    set_ranges(tot);
+    long long cum = before_warp + incl - mine;   // blocks before sequence sbeg
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < K && sbeg + k < S) {
+        const int nb = ceil_div_i(Lr[k], B);
+        if (nb > 0) {
+          const long long lo = cum * Hkv, hi = (cum + nb) * Hkv;
+          for (int kk = 0; kk < NW; ++kk) {
+            const long long uk = warp_u0(kk);
             if (uk >= lo && uk < hi) {
-              loc_s[k] = s;
-              loc_base[k] = lo;
+              loc_s[kk] = sbeg + k;
+              loc_base[kk] = lo;
+              loc_L[kk] = Lr[k];
             }
           }
         }
+        cum += nb;
       }
-      run += chunk_tot;
-      if (run * Hkv > cta_max_u0) break;
+    }
+  } else {
+    // many sequences: a pass for the total, then a chunked scan
+    long long mine = 0;
+    for (int s = threadIdx.x; s < S; s += NT_) {
+      const int nb = seq_blocks<B>(p, s, blockIdx.x == 0);
+      mine += nb;
+      if (nb == 0 && (s % gridDim.x) == blockIdx.x) zero_row(s);
+    }
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, x);
+    if (lane == 0) red[warp] = mine;
+    __syncthreads();
+    long long tot = 0;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) tot += red[k];
+    set_ranges(tot);
+    long long cta_max_u0 = -1;
+    for (int k = 0; k < NW; ++k) cta_max_u0 = max(cta_max_u0, warp_u0(k));
+    if (cta_max_u0 >= 0) {
+      long long run = 0;
+      for (int c0 = 0; c0 < S; c0 += NT_) {
+        const int s = c0 + threadIdx.x;
+        const int L = s < S ? seq_len_clamped<B>(p, s) : 0;
+        const int nb = ceil_div_i(L, B);
+        int incl = nb;
+#pragma unroll
+        for (int x = 1; x < 32; x <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, x);
+          if (lane >= x) incl += v;
+        }
+        __syncthreads();
+        if (lane == 31) red[warp] = incl;
+        __syncthreads();
+        long long before_warp = 0, chunk_tot = 0;
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+          if (k < warp) before_warp += red[k];
+          chunk_tot += red[k];
+        }
+        const long long before = run + before_warp + incl - nb;   // blocks before seq s
+        if (nb > 0) {
+          const long long lo = before * Hkv, hi = (before + nb) * Hkv;
+          for (int kk = 0; kk < NW; ++kk) {
+            const long long uk = warp_u0(kk);
+            if (uk >= lo && uk < hi) {
+              loc_s[kk] = s;
+              loc_base[kk] = lo;
+              loc_L[kk] = L;
+            }
+          }
+        }
+        run += chunk_tot;
+        if (run * Hkv > cta_max_u0) break;
+      }
     }
   }
   __syncthreads();
   if (lane == 0) fence_barrier_init();
   __syncwarp();
+  const bool active = w < w_active;
+  const long long u0 = active ? (w * U) / w_active : 0;
+  const long long u1 = active ? ((w + 1) * U) / w_active : 0;
+  long long *meta = p.meta + w * kMetaWords;
+  if (!active && lane < kMetaWords) meta[lane] = lane == 3 ? U : (lane == 4 ? w_active : 0);
 
   if (!active) return;
 
   // ---- this warp's first tile -----------------------------------------------
   const int s0 = loc_s[warp];
   const long long base0 = loc_base[warp];
-  const int L0 = seq_len_clamped<B>(p, s0);
+  const int L0 = loc_L[warp];
   const int nb0 = ceil_div_i(L0, B);
   const long long r0 = u0 - base0;
   const int h0 = (int)(r0 / nb0);
   const int j0 = (int)(r0 - (long long)h0 * nb0);
+  if (lane < kMetaWords) {
+    const long long seg_lo = base0 + (long long)h0 * nb0;
+    const long long v[kMetaWords] = {u0, seg_lo, seg_lo + nb0, U, w_active, s0, h0, 1};
+    meta[lane] = v[lane];
+  }
   const long long ntiles = u1 - u0;
 
   // ---- issue cursor ---------------------------------------------------------
@@ -895,15 +950,38 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
     if (ti.flags & TF_LAST) {
       const bool complete = seg_from0 && (ti.flags & TF_JEND);
       st.finish(p, ti.s, ti.h, complete, (int)(2 * w + (seg_index == 0 ? 0 : 1)), lane);
-      if (!complete) {
-        const long long lo = ti.u - ti.j;
-        merge_if_last<D, (NT == 0 ? 1 : 4)>(p, ti.s, ti.h, lo, lo + ti.nb, U, w_active, lane);
-      }
       ++seg_index;
     }
     __syncwarp();
     if (i + nstage < ntiles) issue(stage);
   }
+}
+
+// ============================================================================
+// Merge of split segments: one warp per boundary b between warp ranges b-1
+// and b; the warp merges the segment the boundary cuts if it is the first
+// boundary inside that segment.  Launched as a programmatic dependent of the
+// streaming kernel.
+// ============================================================================
+template <int D, int GMAX>
+__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p, int w_total) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const long long b = (long long)blockIdx.x * 4 + (threadIdx.x >> 5) + 1;
+  if (b >= w_total) return;
+  const long long mv = lane < kMetaWords ? __ldcg(p.meta + b * kMetaWords + lane)
+                                         : __ldcg(p.meta + (b - 1) * kMetaWords);
+  const long long u0b = __shfl_sync(0xffffffffu, mv, 0);
+  const long long lo = __shfl_sync(0xffffffffu, mv, 1);
+  const long long hi = __shfl_sync(0xffffffffu, mv, 2);
+  const long long U = __shfl_sync(0xffffffffu, mv, 3);
+  const long long wa = __shfl_sync(0xffffffffu, mv, 4);
+  const int s = (int)__shfl_sync(0xffffffffu, mv, 5);
+  const int h = (int)__shfl_sync(0xffffffffu, mv, 6);
+  const long long active = __shfl_sync(0xffffffffu, mv, 7);
+  const long long u0a = __shfl_sync(0xffffffffu, mv, 8);
+  if (!active || lo >= u0b || lo < u0a) return;
+  merge_parts<D, GMAX>(p, s, h, lo, hi, U, wa, lane);
 }
 
 }  // namespace pa

@@ -59,17 +59,6 @@ std::atomic<int> g_tune_nstage{0};
 std::atomic<int> g_tune_ctas{0};
 std::atomic<int> g_tune_min_tiles{0};
 
-// Per-call epoch for the split-segment tickets: unique, non-zero, < 2^40.
-unsigned long long next_epoch() {
-  static std::atomic<unsigned long long> ctr{0};
-  const unsigned long long mask = (1ull << 40) - 1;
-  unsigned long long e;
-  do {
-    e = (ctr.fetch_add(1) + 1) & mask;
-  } while (e == 0);
-  return e;
-}
-
 struct DecodeLayout {
   int nstage, ctas_per_sm, grid, w_total, min_tiles;
   size_t smem;
@@ -86,7 +75,7 @@ size_t cta_smem(int D, int B, int G, int nstage) {
 }
 
 size_t workspace_for(int w_total, int G, int D, size_t *off_ml, size_t *off_o) {
-  size_t meta = round_up((size_t)w_total * sizeof(unsigned long long), 256);   // tickets
+  size_t meta = round_up((size_t)w_total * pa::kMetaWords * sizeof(long long), 256);
   size_t ml = round_up((size_t)2 * w_total * G * 2 * sizeof(float), 256);
   size_t o = round_up((size_t)2 * w_total * G * D * sizeof(float), 256);
   if (off_ml) *off_ml = meta;
@@ -192,8 +181,7 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   p.q = static_cast<const uint8_t *>(a.q);
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
-  p.tickets = reinterpret_cast<unsigned long long *>(ws + L.off_meta);
-  p.epoch = next_epoch();
+  p.meta = reinterpret_cast<long long *>(ws + L.off_meta);
   p.part_ml = reinterpret_cast<float *>(ws + L.off_ml);
   p.part_o = reinterpret_cast<float *>(ws + L.off_o);
   p.scale_log2 = a.scale * 1.4426950408889634f;
@@ -223,6 +211,23 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   if (cudaLaunchKernelEx(&cfg, kern, kmap, vmap, p) != cudaSuccess) {
     cudaGetLastError();
     return PA_ERR_CUDA;
+  }
+  // Split merge: one warp per boundary between warp ranges, scheduled as the
+  // streaming CTAs retire and released when the streaming grid completes.
+  if (L.w_total > 1) {
+    constexpr int GMAX = NT == 0 ? 1 : 4;
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3((unsigned)((L.w_total - 1 + 3) / 4));
+    mc.blockDim = dim3(128);
+    mc.dynamicSmemBytes = 0;
+    mc.stream = a.stream;
+    mc.attrs = attr;
+    mc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&mc, pa::paged_decode_merge_kernel<D, GMAX>, p, L.w_total) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return PA_ERR_CUDA;
+    }
   }
   return PA_OK;
 }
@@ -434,9 +439,8 @@ int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_
   void *scratch = nullptr;
   const int st = no_alloc_scratch(dev, &scratch);
   if (st != PA_OK) return st;
-  // The scratch needs no clearing: every partial the merge reads is written
-  // by the same call first, and the split-segment counters carry the call's
-  // epoch, so counts left by an earlier call read as zero.  A launch that needs more than
+  // The scratch needs no clearing: every descriptor and partial the merge
+  // reads is written by the same call's streaming kernel first.  A launch that needs more than
   // kNoAllocScratchBytes is refused by launch_decode with PA_ERR_WORKSPACE.
   DecodeArgs a{out,         q,          k_cache,      v_cache,      block_tables,
                context_lens, scale,     num_kv_heads, num_seqs,     num_q_heads,

@@ -155,3 +155,14 @@ def test_device_checks_report_instead_of_faulting(pa, cuda_device):
     pa.pa_copy_blocks(b.k_cache, b.v_cache, torch.tensor([[0, b.num_blocks]], device=dev))
     assert pa.pa_device_error() & pa.DEVERR["copy_pair"]
     assert pa.pa_device_error() == 0
+
+
+def test_many_sequences(pa, cuda_device):
+    """More sequences than one pass of a CTA's threads covers (the chunked
+    scan of the launch plan), short and ragged, some empty."""
+    sh = W.Shape(8, 2, 64, 16, "bf16")
+    rng = np.random.default_rng(17)
+    lens = rng.integers(0, 40, size=1500)
+    b = W.make_decode_batch(sh, lens, seed=21, device=cuda_device, poison="nan")
+    seqs = list(range(0, 1500, 7)) + [1499]
+    check_step(pa, b, seqs=seqs)
