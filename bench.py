@@ -75,18 +75,20 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+def profiled_traffic(bytes_per_launch: float):
+    """DRAM bytes (read + write) per launch from the committed ncu summary,
+    scaled from the profiled launch to this run's launches by algorithmic
+    bytes; None unless the summary was taken on the current kernel source."""
     try:
         text = open(PROFILE_SUMMARY).read()
     except OSError:
         return None
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     m_tr = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
-    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha():
+    m_alg = re.search(r"algorithmic_bytes_of_profiled_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or not m_alg or m_sha.group(1) != kernel_source_sha():
         return None
-    return float(m_tr.group(1))
+    return round(float(m_tr.group(1)) * bytes_per_launch / float(m_alg.group(1)))
 
 
 def measured_hbm_peak():
@@ -315,7 +317,7 @@ def run_b200(args, rank, world, local_rank):
     bytes_launch = float(np.mean(bytes_steps))
     achieved = bytes_launch / (attn_avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
-    traffic = profiled_traffic()
+    traffic = profiled_traffic(bytes_launch)
 
     e2e = None
     if not args.no_e2e:
@@ -356,7 +358,7 @@ def run_b200(args, rank, world, local_rank):
             "decode_tokens_per_s": round(tokens_per_s, 1),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "pa_paged_decode_attention (paged_decode_kernel, split merge fused)",
+                "kernel": "pa_paged_decode_attention (paged_decode_kernel + paged_decode_merge_kernel)",
                 "achieved": round(achieved, 2),
                 "peak": peak,
                 "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6650 GB/s",
