@@ -245,11 +245,11 @@ def run_b200(args, rank, world, local_rank):
     # block manager output for every step, prepared ahead (device-resident arm)
     bm = wl.new_manager(pa)
     seqs = np.arange(S)
-    d_slots, d_tables, d_lens, d_pairs = [], [], [], []
+    d_tables, d_lens, d_pairs = [], [], []
     for step in range(K + Wm):
         slots, pairs = bm.append_slots(seqs)
         tables, lens = bm.block_tables(seqs, wl.maxb)
-        d_slots.append(torch.as_tensor(slots, device=dev))
+
         d_tables.append(torch.as_tensor(tables, device=dev))
         d_lens.append(torch.as_tensor(lens, device=dev))
         d_pairs.append(torch.as_tensor(pairs, device=dev) if len(pairs) else None)
@@ -257,8 +257,8 @@ def run_b200(args, rank, world, local_rank):
     maxctx = wl.maxb * B
     ws = pa.alloc_workspace(S, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, B, maxctx, dev)
     out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
-    # kernels launched per timed step: reshape_and_cache + decode attention,
-    # plus copy_blocks on steps with copy-on-write pairs
+    # kernels launched per timed step: the fused decode step and its split
+    # merge, plus copy_blocks on steps with copy-on-write pairs
     timed_launches = sum(2 + (d_pairs[Wm + k] is not None) for k in range(K))
 
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -267,12 +267,12 @@ def run_b200(args, rank, world, local_rank):
     def step(i, timed_idx=None):
         if d_pairs[i] is not None:
             pa.pa_copy_blocks(b.k_cache, b.v_cache, d_pairs[i])
-        pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, d_slots[i])
         if timed_idx is not None:
             ev_a[timed_idx].record(stream)
-        pa.pa_paged_decode_attention(out, b.q, b.k_cache, b.v_cache, d_tables[i], d_lens[i],
-                                     wl.scale, sh.num_kv_heads, max_context_len=maxctx,
-                                     workspace=ws)
+        # fused: the newest token's cache write + decode attention (+ split merge)
+        pa.pa_decode_step(out, b.q, b.k_new, b.v_new, b.k_cache, b.v_cache, d_tables[i],
+                          d_lens[i], wl.scale, sh.num_kv_heads, max_context_len=maxctx,
+                          workspace=ws)
         if timed_idx is not None:
             ev_b[timed_idx].record(stream)
 
@@ -351,14 +351,14 @@ def run_b200(args, rank, world, local_rank):
                 "mean_context_len": float(np.mean(wl.lens0)) + Wm + (K - 1) / 2,
                 "parallelism": f"dp{world} (independent batches, no collective on the data path)",
                 "l2": "inputs larger than L2: %.2f GB of KV read per step, no flush" % (bytes_launch / 1e9),
-                "step": "host block manager (prepared ahead) -> reshape_and_cache -> paged decode attention (split merge fused)",
+                "step": "host block manager (prepared ahead) -> copy_blocks if any -> pa_decode_step (cache write of the new token + paged decode attention) -> split merge",
             },
             "pct_of_measured_hbm_peak": round(100.0 * value / peak / world, 2),
             "pct_of_nominal_8tbs": round(100.0 * value / 8000.0 / world, 2),
             "decode_tokens_per_s": round(tokens_per_s, 1),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "pa_paged_decode_attention (paged_decode_kernel + paged_decode_merge_kernel)",
+                "kernel": "pa_decode_step (paged_decode_kernel with the newest token's cache write, + paged_decode_merge_kernel)",
                 "achieved": round(achieved, 2),
                 "peak": peak,
                 "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6650 GB/s",
@@ -378,8 +378,12 @@ def run_b200(args, rank, world, local_rank):
 
 
 def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
-    """Same metric through the public API from pinned host buffers: block
-    manager on the host, H2D of the step's inputs, kernels, D2H of the output."""
+    """Same metric through the public API from pinned host buffers: per step,
+    the host block manager reserves the slots, the step's inputs (q, new K/V,
+    slots, block tables, lengths) go host -> device, the library's kernels
+    run, and the output comes back device -> host.  Three streams (upload,
+    compute, download) and three buffer sets let step i+1's upload and step
+    i-1's download overlap step i's kernels; events order every reuse."""
     import torch
     import torch.distributed as dist
     sh = wl.shape
@@ -387,53 +391,72 @@ def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
     b = wl.batch
     seqs = np.arange(S)
     bm = wl.new_manager(pa)
-    # host copies of the step's inputs (values reused each step)
-    h_q = [b.q.cpu().pin_memory() for _ in range(2)]
-    h_k = [b.k_new.cpu().pin_memory() for _ in range(2)]
-    h_v = [b.v_new.cpu().pin_memory() for _ in range(2)]
-    h_slots = [torch.empty(S, dtype=torch.int64).pin_memory() for _ in range(2)]
-    h_tables = [torch.empty(S, wl.maxb, dtype=torch.int32).pin_memory() for _ in range(2)]
-    h_lens = [torch.empty(S, dtype=torch.int32).pin_memory() for _ in range(2)]
+    NBUF = 3
+    h_q = [b.q.cpu().pin_memory() for _ in range(NBUF)]
+    h_k = [b.k_new.cpu().pin_memory() for _ in range(NBUF)]
+    h_v = [b.v_new.cpu().pin_memory() for _ in range(NBUF)]
+    h_slots = [torch.empty(S, dtype=torch.int64).pin_memory() for _ in range(NBUF)]
+    h_tables = [torch.empty(S, wl.maxb, dtype=torch.int32).pin_memory() for _ in range(NBUF)]
+    h_lens = [torch.empty(S, dtype=torch.int32).pin_memory() for _ in range(NBUF)]
     h_out = [torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32).pin_memory()
-             for _ in range(2)]
-    d_q = torch.empty_like(b.q)
-    d_k = torch.empty_like(b.k_new)
-    d_v = torch.empty_like(b.v_new)
-    d_slots = torch.empty(S, dtype=torch.int64, device=dev)
-    d_tables = torch.empty(S, wl.maxb, dtype=torch.int32, device=dev)
-    d_lens = torch.empty(S, dtype=torch.int32, device=dev)
-    d_out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+             for _ in range(NBUF)]
+    d_q = [torch.empty_like(b.q) for _ in range(NBUF)]
+    d_k = [torch.empty_like(b.k_new) for _ in range(NBUF)]
+    d_v = [torch.empty_like(b.v_new) for _ in range(NBUF)]
+    d_slots = [torch.empty(S, dtype=torch.int64, device=dev) for _ in range(NBUF)]
+    d_tables = [torch.empty(S, wl.maxb, dtype=torch.int32, device=dev) for _ in range(NBUF)]
+    d_lens = [torch.empty(S, dtype=torch.int32, device=dev) for _ in range(NBUF)]
+    d_pairs = [torch.empty(S, 2, dtype=torch.int64, device=dev) for _ in range(NBUF)]
+    h_pairs = [torch.empty(S, 2, dtype=torch.int64).pin_memory() for _ in range(NBUF)]
+    d_out = [torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+             for _ in range(NBUF)]
     maxctx = wl.maxb * B
     ws = pa.alloc_workspace(S, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, B, maxctx, dev)
-    done = [None, None]
-    h2d = sum(t[0].numel() * t[0].element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_lens))
+    s_up, s_cmp, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [None] * NBUF    # upload of the set done
+    ev_cmp = [None] * NBUF   # kernels that read the set's inputs / write its output done
+    ev_dn = [None] * NBUF    # download of the set's output done
+    h2d = sum(t[0].numel() * t[0].element_size() for t in (h_q, h_k, h_v, h_tables, h_lens))
     d2h = h_out[0].numel() * 4
 
     def one(i):
-        j = i % 2
-        if done[j] is not None:
-            done[j].synchronize()          # buffers of step i-2 are free again
+        j = i % NBUF
+        if ev_up[j] is not None:
+            ev_up[j].synchronize()             # host buffers of set j are free again
         slots, pairs = bm.append_slots(seqs)
         h_slots[j].numpy()[:] = slots
         tables, lens = bm.block_tables(seqs, wl.maxb)
         h_tables[j].numpy()[:] = tables
         h_lens[j].numpy()[:] = lens
-        d_q.copy_(h_q[j], non_blocking=True)
-        d_k.copy_(h_k[j], non_blocking=True)
-        d_v.copy_(h_v[j], non_blocking=True)
-        d_slots.copy_(h_slots[j], non_blocking=True)
-        d_tables.copy_(h_tables[j], non_blocking=True)
-        d_lens.copy_(h_lens[j], non_blocking=True)
-        if len(pairs):
-            pa.pa_copy_blocks(b.k_cache, b.v_cache, torch.as_tensor(pairs).to(dev, non_blocking=True))
-        pa.pa_reshape_and_cache(d_k, d_v, b.k_cache, b.v_cache, d_slots)
-        pa.pa_paged_decode_attention(d_out, d_q, b.k_cache, b.v_cache, d_tables, d_lens,
-                                     wl.scale, sh.num_kv_heads, max_context_len=maxctx,
-                                     workspace=ws)
-        h_out[j].copy_(d_out, non_blocking=True)
-        ev = torch.cuda.Event()
-        ev.record()
-        done[j] = ev
+        npairs = len(pairs)
+        if npairs:
+            h_pairs[j].numpy()[:npairs] = pairs
+        with torch.cuda.stream(s_up):
+            if ev_cmp[j] is not None:
+                s_up.wait_event(ev_cmp[j])     # device inputs of set j no longer read
+            for d, h in ((d_q[j], h_q[j]), (d_k[j], h_k[j]), (d_v[j], h_v[j]),
+                         (d_tables[j], h_tables[j]), (d_lens[j], h_lens[j])):
+                d.copy_(h, non_blocking=True)
+            if npairs:
+                d_pairs[j][:npairs].copy_(h_pairs[j][:npairs], non_blocking=True)
+            ev_up[j] = torch.cuda.Event()
+            ev_up[j].record(s_up)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_up[j])
+            if ev_dn[j] is not None:
+                s_cmp.wait_event(ev_dn[j])     # output of set j downloaded
+            if npairs:
+                pa.pa_copy_blocks(b.k_cache, b.v_cache, d_pairs[j][:npairs])
+            pa.pa_decode_step(d_out[j], d_q[j], d_k[j], d_v[j], b.k_cache, b.v_cache,
+                              d_tables[j], d_lens[j], wl.scale, sh.num_kv_heads,
+                              max_context_len=maxctx, workspace=ws)
+            ev_cmp[j] = torch.cuda.Event()
+            ev_cmp[j].record(s_cmp)
+        with torch.cuda.stream(s_dn):
+            s_dn.wait_event(ev_cmp[j])
+            h_out[j].copy_(d_out[j], non_blocking=True)
+            ev_dn[j] = torch.cuda.Event()
+            ev_dn[j].record(s_dn)
 
     for i in range(Wm):
         one(i)
@@ -451,7 +474,8 @@ def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
     return {"value": round(bytes_all / dt_max / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(dt_max * 1e3 / K, 4),
-            "timing": "host wall clock, synchronize on both sides, max over ranks"}
+            "timing": "host wall clock, synchronize on both sides, max over ranks; "
+                      "upload / compute / download on three streams, three buffer sets"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)

@@ -142,6 +142,32 @@ int pa_paged_decode_attention(float *out, const void *q, const void *k_cache,
                               pa_stream_t stream);
 
 /*
+ * One decode step fused into one launch: the cache write of every sequence's
+ * newest token (as pa_reshape_and_cache would do it) and the decode attention
+ * over all of its tokens (as pa_paged_decode_attention).  Follows the same
+ * pages: [P1] section 2 (on-demand allocation of the new token's slot; the
+ * kernel that reads K/V through the block table for the new token).
+ *
+ *   k_new, v_new  dtype [num_seqs, num_kv_heads, head_dim] (device): the K/V
+ *                 of token L-1 of each sequence (L = context_lens[s]); it is
+ *                 stored at position L-1 of the sequence's block table, i.e.
+ *                 in block block_tables[s][(L-1) / B] at offset (L-1) % B,
+ *                 and attention uses it directly.  Sequences with L == 0 have
+ *                 no new token and get a zero row.
+ *   k_cache, v_cache are written (that one slot per sequence and kv head).
+ * All other arguments as for pa_paged_decode_attention.  The result equals
+ * pa_reshape_and_cache with slot_mapping[s] = that position, followed by
+ * pa_paged_decode_attention; the block holding position L-1 must be the
+ * sequence's own (not shared: copy it with pa_copy_blocks first).
+ */
+int pa_decode_step(float *out, const void *q, const void *k_new, const void *v_new,
+                   void *k_cache, void *v_cache, const int32_t *block_tables,
+                   const int32_t *context_lens, float scale, int num_kv_heads, int num_seqs,
+                   int num_q_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                   int max_context_len, int num_blocks, pa_dtype dtype, void *workspace,
+                   size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * Allocation-free variant of pa_paged_decode_attention (no counterpart in the
  * pages: an integration convenience).  Same arguments, same result, but no
  * workspace argument: the split-context scratch lives in a fixed array of

@@ -70,6 +70,8 @@ def _declare(L):
                                             i32, i32, i32, i32, vp, sz, vp]),
         "pa_paged_decode_attention_no_alloc": (i32, [vp, vp, vp, vp, vp, vp, f32, i32, i32, i32,
                                                      i32, i32, i32, i32, i32, i32, vp]),
+        "pa_decode_step": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32,
+                                 i32, i32, i32, i32, vp, sz, vp]),
         "pa_decode_tuning": (i32, [i32, i32, i32]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
         "pa_device_error": (i32, [c.POINTER(c.c_uint), i32]),
@@ -223,6 +225,39 @@ def pa_paged_decode_attention_no_alloc(out, q, k_cache, v_cache, block_tables, c
         _dev(context_lens, "context_lens", torch.int32), float(scale), Hkv, S, Hq, D, B, maxb,
         int(max_context_len), NB, _dtype_code(k_cache), _stream(stream))
     _check(st, "pa_paged_decode_attention_no_alloc")
+    return out
+
+
+def pa_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale,
+                   num_kv_heads, max_context_len=None, workspace=None, stream=None):
+    """One fused decode step: store each sequence's newest token (k_new/v_new
+    [S, Hkv, D]) at position L-1 of its block table and attend over all L
+    tokens; equals pa_reshape_and_cache followed by pa_paged_decode_attention."""
+    torch = _torch()
+    S, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    if Hkv != num_kv_heads or D2 != D:
+        raise ValueError("q / cache shapes disagree")
+    if tuple(k_new.shape) != (S, Hkv, D) or tuple(v_new.shape) != (S, Hkv, D):
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim]")
+    if tuple(out.shape) != (S, Hq, D):
+        raise ValueError("out must be [num_seqs, num_q_heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables [S, max_blocks] / context_lens [S] expected")
+    maxb = int(block_tables.shape[1])
+    if max_context_len is None:
+        max_context_len = maxb * B
+    if workspace is None:
+        workspace = alloc_workspace(S, Hq, Hkv, D, B, max_context_len, q.device)
+    dt = k_cache.dtype
+    st = lib().pa_decode_step(
+        _dev(out, "out", torch.float32), _dev(q, "q", dt), _dev(k_new, "k_new", dt),
+        _dev(v_new, "v_new", dt), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", dt),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), float(scale), Hkv, S, Hq, D, B, maxb,
+        int(max_context_len), NB, _dtype_code(k_cache), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "pa_decode_step")
     return out
 
 

@@ -59,16 +59,24 @@ enum : int {
   TF_J0 = 4,      // logical block 0 of the segment
   TF_JEND = 8,    // last logical block of the segment
   TF_SKIP = 16,   // block id out of range: no data, contributes nothing
+  TF_NEWTOK = 32, // holds the sequence's newest token, which this call also writes
 };
 
 struct TileInfo {
-  int s, h, j, valid, flags, nb;
+  int s, h, j, valid, flags, nb, blk, pad;
   long long u;   // global tile index
 };
 
 struct DecodeParams {
   float *out;
   const uint8_t *q;
+  // Fused cache write (decode step): the newest token of every sequence comes
+  // from k_new / v_new [S, Hkv, D] and is also stored into the pool.  Null
+  // for attention alone.
+  const uint8_t *k_new;
+  const uint8_t *v_new;
+  uint8_t *k_cache_w;
+  uint8_t *v_cache_w;
   const int32_t *block_tables;
   const int32_t *context_lens;
   long long *meta;     // [w_total][kMetaWords]: each warp's range and first segment
@@ -636,6 +644,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   constexpr int STAGE = 2 * TILE;
   const int G = p.group;
   const int qbytes = G * D * 2;
+  const int qstride = qbytes + 4 * D;   // query rows, then the new K and V rows
   const int nstage = p.nstage;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.num_seqs, Hkv = p.num_kv_heads;
@@ -645,11 +654,11 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // per-warp regions
   uint8_t *stages = smem + (size_t)warp * nstage * STAGE;
-  uint8_t *qslots = smem + (size_t)NW * nstage * STAGE + (size_t)warp * nstage * qbytes;
-  TileInfo *info = reinterpret_cast<TileInfo *>(smem + (size_t)NW * nstage * (STAGE + qbytes)) +
+  uint8_t *qslots = smem + (size_t)NW * nstage * STAGE + (size_t)warp * nstage * qstride;
+  TileInfo *info = reinterpret_cast<TileInfo *>(smem + (size_t)NW * nstage * (STAGE + qstride)) +
                    warp * nstage;
   uint64_t *bars = reinterpret_cast<uint64_t *>(
-                       smem + (size_t)NW * nstage * (STAGE + qbytes + sizeof(TileInfo))) +
+                       smem + (size_t)NW * nstage * (STAGE + qstride + sizeof(TileInfo))) +
                    warp * nstage;
 
   __shared__ long long red[NW];
@@ -882,13 +891,17 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
         flags |= TF_SKIP;
         flag_error(PA_DEVERR_BLOCK_ID);
       }
+      if (ok && p.k_new != nullptr && j == cur.nb - 1) flags |= TF_NEWTOK;
       const int valid = min(B, cur.L - j * B);
       TileInfo ti;
       ti.s = cur.s; ti.h = h; ti.j = j; ti.valid = valid; ti.flags = flags;
       ti.nb = cur.nb;
+      ti.blk = id;
+      ti.pad = 0;
       ti.u = u0 + issued;
       info[stage] = ti;
-      const uint32_t bytes = (ok ? STAGE : 0) + ((flags & TF_FIRST) ? qbytes : 0);
+      const uint32_t bytes = (ok ? STAGE : 0) + ((flags & TF_FIRST) ? qbytes : 0) +
+                             ((flags & TF_NEWTOK) ? 4 * D : 0);
       uint64_t *bar = &bars[stage];
       if (bytes) {
         fence_proxy_async_smem();
@@ -903,9 +916,14 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
           }
         }
         if (flags & TF_FIRST)
-          bulk_load(qslots + (size_t)stage * qbytes,
+          bulk_load(qslots + (size_t)stage * qstride,
                     qbase + ((int64_t)cur.s * p.num_q_heads + (int64_t)h * G) * (D * 2), qbytes,
                     bar);
+        if (flags & TF_NEWTOK) {
+          const int64_t row = ((int64_t)cur.s * Hkv + h) * (D * 2);
+          bulk_load(qslots + (size_t)stage * qstride + qbytes, p.k_new + row, D * 2, bar);
+          bulk_load(qslots + (size_t)stage * qstride + qbytes + 2 * D, p.v_new + row, D * 2, bar);
+        }
       } else {
         mbar_arrive(bar);
       }
@@ -936,8 +954,25 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
     const TileInfo ti = info[stage];
     if (ti.flags & TF_FIRST) {
       st.reset();
-      st.load_q(qslots + (size_t)stage * qbytes, G, lane);
+      st.load_q(qslots + (size_t)stage * qstride, G, lane);
       seg_from0 = (ti.flags & TF_J0) != 0;
+    }
+    if (ti.flags & TF_NEWTOK) {
+      // the newest token: patch its K and V rows into the staged tile (the
+      // pool still holds whatever was in that slot) and store them in the pool
+      constexpr int CH = D / 8;   // 16-byte chunks per row
+      const int r = ti.valid - 1;
+      if (lane < 2 * CH) {
+        const int isv = lane / CH, c = lane % CH;
+        const uint4 v = *reinterpret_cast<const uint4 *>(qslots + (size_t)stage * qstride +
+                                                         qbytes + isv * (2 * D) + c * 16);
+        uint8_t *tile = stages + (size_t)stage * STAGE + isv * TILE;
+        *reinterpret_cast<uint4 *>(tile + swz<B>(c >> 3, r, c & 7)) = v;
+        uint8_t *pool = isv ? p.v_cache_w : p.k_cache_w;
+        *reinterpret_cast<uint4 *>(pool + (((int64_t)ti.blk * Hkv + ti.h) * B + r) * (D * 2) +
+                                   c * 16) = v;
+      }
+      __syncwarp();
     }
     if (!(ti.flags & TF_SKIP)) {
       const uint8_t *ks = stages + (size_t)stage * STAGE;

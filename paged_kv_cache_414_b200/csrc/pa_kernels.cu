@@ -66,7 +66,8 @@ struct DecodeLayout {
 };
 
 size_t stage_bytes(int D, int B, int G) {
-  return 2 * (size_t)B * D * 2 + (size_t)G * D * 2 + sizeof(pa::TileInfo) + sizeof(uint64_t);
+  return 2 * (size_t)B * D * 2 + (size_t)G * D * 2 + 4 * (size_t)D + sizeof(pa::TileInfo) +
+         sizeof(uint64_t);
 }
 
 // Shared-memory need of one CTA with `nstage` stages per warp.
@@ -138,6 +139,7 @@ bool encode_pool_map(CUtensorMap *m, const void *base, long long rows, int D, in
 struct DecodeArgs {
   float *out;
   const void *q, *k_cache, *v_cache;
+  const void *k_new, *v_new;   // non-null: fused decode step (cache write of the newest token)
   const int32_t *block_tables, *context_lens;
   float scale;
   int num_kv_heads, num_seqs, num_q_heads, head_dim, block_size, max_blocks, num_blocks;
@@ -179,6 +181,10 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   pa::DecodeParams p;
   p.out = a.out;
   p.q = static_cast<const uint8_t *>(a.q);
+  p.k_new = static_cast<const uint8_t *>(a.k_new);
+  p.v_new = static_cast<const uint8_t *>(a.v_new);
+  p.k_cache_w = static_cast<uint8_t *>(const_cast<void *>(a.k_cache));
+  p.v_cache_w = static_cast<uint8_t *>(const_cast<void *>(a.v_cache));
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
   p.meta = reinterpret_cast<long long *>(ws + L.off_meta);
@@ -367,10 +373,46 @@ int pa_paged_decode_attention(float *out, const void *q, const void *k_cache,
   if (current_device(&dev) != PA_OK || dev >= kMaxDevices) return PA_ERR_CUDA;
   const int sms = sm_count(dev);
   if (sms <= 0) return PA_ERR_CUDA;
-  DecodeArgs a{out,         q,          k_cache,      v_cache,      block_tables,
-               context_lens, scale,     num_kv_heads, num_seqs,     num_q_heads,
-               head_dim,    block_size, max_blocks_per_seq, num_blocks, workspace,
-               workspace_bytes, (cudaStream_t)stream};
+  DecodeArgs a{out,          q,           k_cache,      v_cache,      nullptr,
+               nullptr,      block_tables, context_lens, scale,        num_kv_heads,
+               num_seqs,     num_q_heads, head_dim,     block_size,   max_blocks_per_seq,
+               num_blocks,   workspace,   workspace_bytes, (cudaStream_t)stream};
+  if (dtype == PA_BF16) return dispatch_shape<__nv_bfloat16>(a, dev, sms);
+  return dispatch_shape<__half>(a, dev, sms);
+}
+
+int pa_decode_step(float *out, const void *q, const void *k_new, const void *v_new,
+                   void *k_cache, void *v_cache, const int32_t *block_tables,
+                   const int32_t *context_lens, float scale, int num_kv_heads, int num_seqs,
+                   int num_q_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                   int max_context_len, int num_blocks, pa_dtype dtype, void *workspace,
+                   size_t workspace_bytes, pa_stream_t stream) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || head_dim <= 0 || block_size <= 0)
+    return PA_ERR_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_ARG;
+  if (!supported_shape(head_dim, block_size) || num_q_heads / num_kv_heads > 16)
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
+      (long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_ARG;
+  if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+  if (!out || !q || !k_new || !v_new || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+      !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_tables, 4) ||
+      !aligned(context_lens, 4))
+    return PA_ERR_ARG;
+  if (!workspace || !aligned(workspace, 256)) return PA_ERR_WORKSPACE;
+  int dev;
+  if (current_device(&dev) != PA_OK || dev >= kMaxDevices) return PA_ERR_CUDA;
+  const int sms = sm_count(dev);
+  if (sms <= 0) return PA_ERR_CUDA;
+  DecodeArgs a{out,          q,           k_cache,      v_cache,      k_new,
+               v_new,        block_tables, context_lens, scale,        num_kv_heads,
+               num_seqs,     num_q_heads, head_dim,     block_size,   max_blocks_per_seq,
+               num_blocks,   workspace,   workspace_bytes, (cudaStream_t)stream};
   if (dtype == PA_BF16) return dispatch_shape<__nv_bfloat16>(a, dev, sms);
   return dispatch_shape<__half>(a, dev, sms);
 }
@@ -442,10 +484,10 @@ int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_
   // The scratch needs no clearing: every descriptor and partial the merge
   // reads is written by the same call's streaming kernel first.  A launch that needs more than
   // kNoAllocScratchBytes is refused by launch_decode with PA_ERR_WORKSPACE.
-  DecodeArgs a{out,         q,          k_cache,      v_cache,      block_tables,
-               context_lens, scale,     num_kv_heads, num_seqs,     num_q_heads,
-               head_dim,    block_size, max_blocks_per_seq, num_blocks, scratch,
-               kNoAllocScratchBytes, (cudaStream_t)stream};
+  DecodeArgs a{out,          q,           k_cache,      v_cache,      nullptr,
+               nullptr,      block_tables, context_lens, scale,        num_kv_heads,
+               num_seqs,     num_q_heads, head_dim,     block_size,   max_blocks_per_seq,
+               num_blocks,   scratch,     kNoAllocScratchBytes, (cudaStream_t)stream};
   if (dtype == PA_BF16) return dispatch_shape<__nv_bfloat16>(a, dev, sms);
   return dispatch_shape<__half>(a, dev, sms);
 }

@@ -60,6 +60,25 @@ class Expected:
                                              sh.num_kv_heads, B, sh.dtype)
 
 
+def library_fused_step(pa, batch: W.DecodeBatch):
+    """One decode step through the fused entry point pa_decode_step (cache
+    write of the newest token + attention in one launch).  Returns (tables, out)."""
+    sh = batch.shape
+    S = batch.num_seqs
+    bm = pa.BlockManager(batch.num_blocks, sh.block_size, batch.free_order)
+    for s in range(S):
+        bm.allocate(s, int(batch.context_lens[s]))
+    tables, lens = bm.block_tables(np.arange(S), batch.max_blocks_per_seq)
+    dev = batch.q.device
+    out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+    pa.pa_decode_step(out, batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache,
+                      torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev),
+                      batch.scale, sh.num_kv_heads,
+                      max_context_len=int(batch.context_lens.max(initial=0)))
+    torch.cuda.synchronize()
+    return tables, out
+
+
 def library_step(pa, batch: W.DecodeBatch, tuning=None):
     """One decode step through the library: native manager slots, cache write,
     attention.  Returns (slots, tables, out)."""

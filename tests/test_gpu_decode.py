@@ -166,3 +166,42 @@ def test_many_sequences(pa, cuda_device):
     b = W.make_decode_batch(sh, lens, seed=21, device=cuda_device, poison="nan")
     seqs = list(range(0, 1500, 7)) + [1499]
     check_step(pa, b, seqs=seqs)
+
+
+FUSED_SHAPES = [("bf16", 128, 16, 32, 8), ("f16", 128, 16, 8, 8), ("bf16", 64, 32, 16, 2),
+                ("f16", 64, 16, 4, 4), ("bf16", 128, 32, 64, 8)]
+
+
+@pytest.mark.parametrize("dtype,D,B,Hq,Hkv", FUSED_SHAPES)
+def test_fused_decode_step(pa, cuda_device, dtype, D, B, Hq, Hkv):
+    """pa_decode_step (newest token's cache write + attention in one launch)
+    against the oracle: the pool bit for bit, the output within tolerance."""
+    from parity import library_fused_step
+    sh = W.Shape(Hq, Hkv, D, B, dtype)
+    lens = [1, 0, 15, 16, 17, 33, 100, 257, 1000, 2048, 3001, 7]
+    b = W.make_decode_batch(sh, lens, seed=D + B + Hq + 1, device=cuda_device, poison="nan")
+    exp = Expected(b)
+    tables, out = library_fused_step(pa, b)
+    idx = torch.as_tensor(exp.blocks, device=cuda_device)
+    assert np.array_equal(W.bits(b.k_cache.index_select(0, idx)), exp.k_after)
+    assert np.array_equal(W.bits(b.v_cache.index_select(0, idx)), exp.v_after)
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    assert max_abs_err(got, exp.out) <= TOL
+    assert (got[1] == 0).all()
+    assert pa.pa_device_error() == 0
+
+
+def test_fused_step_equals_two_calls(pa, cuda_device):
+    """The fused step gives bit for bit the result of reshape_and_cache
+    followed by decode attention."""
+    from parity import library_fused_step
+    sh = W.Shape(32, 8, 128, 16, "bf16")
+    rng = np.random.default_rng(8)
+    lens = rng.integers(1, 2500, size=64)
+    b1 = W.make_decode_batch(sh, lens, seed=6, device=cuda_device)
+    b2 = W.make_decode_batch(sh, lens, seed=6, device=cuda_device)
+    _, _, out1 = library_step(pa, b1)
+    _, out2 = library_fused_step(pa, b2)
+    assert torch.equal(out1, out2)
+    assert torch.equal(b1.k_cache, b2.k_cache) and torch.equal(b1.v_cache, b2.v_cache)

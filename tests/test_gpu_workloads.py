@@ -50,7 +50,8 @@ def test_peaked_long_context_follows_the_hot_tokens(pa, cuda_device):
     assert err <= TOL
 
 
-def test_parallel_sampling_copy_on_write(pa, cuda_device):
+@pytest.mark.parametrize("fused", [False, True])
+def test_parallel_sampling_copy_on_write(pa, cuda_device, fused):
     wl = W.cow_workload(device=cuda_device)
     sh = wl.shape
     B = sh.block_size
@@ -98,15 +99,21 @@ def test_parallel_sampling_copy_on_write(pa, cuda_device):
         # device: copy-on-write copies before the step's cache write
         if len(npairs):
             pa.pa_copy_blocks(k, v, torch.as_tensor(npairs, device=dev))
-        pa.pa_reshape_and_cache(kn, vn, k, v, torch.as_tensor(nslots, device=dev))
+        tables, lens = nbm.block_tables(seqs, cap)
+        out = torch.empty(S, sh.num_q_heads, sh.head_dim, device=dev)
+        scale = 1.0 / np.sqrt(sh.head_dim)
+        if fused:
+            pa.pa_decode_step(out, q, kn, vn, k, v, torch.as_tensor(tables, device=dev),
+                              torch.as_tensor(lens, device=dev), scale, sh.num_kv_heads,
+                              max_context_len=cap * B, workspace=ws)
+        else:
+            pa.pa_reshape_and_cache(kn, vn, k, v, torch.as_tensor(nslots, device=dev))
+            pa.pa_paged_decode_attention(out, q, k, v, torch.as_tensor(tables, device=dev),
+                                         torch.as_tensor(lens, device=dev), scale,
+                                         sh.num_kv_heads, max_context_len=cap * B, workspace=ws)
         if opairs:
             OC.copy_blocks(kb, vb, np.array(opairs))
         OC.reshape_and_cache(knb, vnb, kb, vb, np.array(oslots), B)
-        tables, lens = nbm.block_tables(seqs, cap)
-        out = torch.empty(S, sh.num_q_heads, sh.head_dim, device=dev)
-        pa.pa_paged_decode_attention(out, q, k, v, torch.as_tensor(tables, device=dev),
-                                     torch.as_tensor(lens, device=dev), 1.0 / np.sqrt(sh.head_dim),
-                                     sh.num_kv_heads, max_context_len=cap * B, workspace=ws)
         if step in (0, 1, wl.steps - 1):
             torch.cuda.synchronize()
             assert np.array_equal(W.bits(k), kb) and np.array_equal(W.bits(v), vb)
