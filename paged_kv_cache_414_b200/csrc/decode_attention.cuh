@@ -16,10 +16,12 @@
 // softmax state per segment; a segment that lies wholly inside one warp's
 // range is written to `out` directly, a segment cut by range boundaries
 // leaves one (max, sum, accumulator) partial per warp that touched it
-// (split context).  A small merge kernel, launched as a programmatic
-// dependent so it starts as soon as the last streaming warp is done, combines
-// the partials: one warp per boundary between warp ranges.  The streaming
-// kernel itself never waits, fences or takes an atomic.
+// (split context), plus an 8-word descriptor of its range and first segment.
+// A small merge kernel, launched as a programmatic dependent so its CTAs are
+// resident and waiting when the streaming grid completes, combines the
+// partials: one warp per (boundary between warp ranges, group of heads).
+// The streaming kernel itself never waits on another warp, fences or takes
+// an atomic.
 //
 // Data movement.  Each warp owns a ring of `nstage` shared-memory stages and
 // issues its own copies: one 2-D TMA box per 64 head-dim columns of the K
@@ -83,7 +85,7 @@ struct DecodeParams {
   float *part_ml;      // [2 * w_total][G][2]   (max in log2 units, sum)
   float *part_o;       // [2 * w_total][G][D]
   float scale_log2;    // scale * log2(e)
-  int num_seqs, num_q_heads, num_kv_heads, group;
+  int num_seqs, num_q_heads, num_kv_heads, group, head_dim;
   int max_blocks, num_blocks;
   int nstage;
   int min_tiles;       // fewest tiles a warp is given
@@ -508,101 +510,154 @@ __device__ __forceinline__ long long part_slot(long long c, long long lo, long l
   return (lo <= warp_start(c, U, wa)) ? 2 * c : 2 * c + 1;
 }
 
-// Merge all partials of the split segment (s, h) = tiles [lo, hi): with
-// M = max_i m_i, out = sum_i 2^(m_i - M) acc_i / sum_i 2^(m_i - M) l_i.
-template <int D, int GMAX>
-__device__ void merge_parts(const DecodeParams &p, int s, int h, long long lo, long long hi,
-                            long long U, long long wa, int lane) {
-  constexpr int VPL = D / 32;
-  const long long c_lo = warp_of(lo, U, wa), c_hi = warp_of(hi - 1, U, wa);
-  const long long n = c_hi - c_lo + 1;
-  const int G = p.group;
-  float *dst = p.out + ((int64_t)s * p.num_q_heads + (int64_t)h * G) * D + lane * VPL;
-  using VecT = typename std::conditional<VPL == 4, float4, float2>::type;
-  // Heads in chunks of GMAX.  Lane k reads partial k's (max, sum); the
-  // accumulators are read UNR partials at a time with every load issued
-  // before any is used, so the L2 latency is paid once per UNR partials.
-  constexpr int UNR = 4;
-  for (int g0 = 0; g0 < G; g0 += GMAX) {
-    float M[GMAX], den[GMAX], num[GMAX][VPL];
-#pragma unroll
-    for (int g = 0; g < GMAX; ++g) {
-      M[g] = -INFINITY;
-      den[g] = 0.f;
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) num[g][v] = 0.f;
+// ============================================================================
+// Launch plan, computed by every CTA from the context lengths alone: the total
+// number of tiles U = Hkv * sum_s ceil(L_s / B), the number of active warps
+// (at most w_total, at least p.min_tiles tiles each), and for each of NQ query
+// tiles query(k, U, w_active) (negative = none) the sequence holding it, the
+// sequence's first tile and its (clamped) length.  With zero_rows set, the
+// output rows of empty sequences are zeroed (each by one CTA) and bad lengths
+// reported.  All threads of the CTA must call it; it ends with __syncthreads.
+// ============================================================================
+template <int B, int NW, typename Query>
+__device__ void cta_plan(const DecodeParams &p, long long w_total, Query query, bool zero_rows,
+                         long long *red, int *loc_s, long long *loc_base, int *loc_L,
+                         long long &U, long long &w_active) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int S = p.num_seqs, Hkv = p.num_kv_heads;
+  constexpr int NT_ = NW * 32;   // threads per CTA
+  constexpr int KMAX = 8;   // sequences per thread on the one-pass path
+  U = 0;
+  w_active = 0;
+  auto set_ranges = [&](long long tot) {
+    U = tot * Hkv;
+    w_active = 0;
+    if (U > 0) {
+      w_active = (U + p.min_tiles - 1) / p.min_tiles;
+      if (w_active > w_total) w_active = w_total;
     }
-    for (long long k0 = 0; k0 < n; k0 += 32) {
-      const long long k = k0 + lane;
-      const bool ok = k < n;
-      const long long c = c_lo + k;
-      const long long slot = ok ? part_slot(c, lo, U, wa) : 0;
-      const int cnt = (int)((n - k0) < 32 ? (n - k0) : 32);
-      float wk[GMAX];
+  };
+  auto warp_u0 = [&](int k) -> long long { return query(k, U, w_active); };
+  const int D = p.head_dim;
+  auto zero_row = [&](int s) {   // empty sequence: zero output rows
+    if (!zero_rows) return;
+    float4 *row = reinterpret_cast<float4 *>(p.out + (int64_t)s * p.num_q_heads * D);
+    for (int k = 0; k < p.num_q_heads * D / 4; ++k) row[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  const int cap = p.max_blocks * B;
+  if (S <= NT_ * KMAX) {
+    // one pass: thread t owns sequences [t*K, t*K + K)
+    const int K = (S + NT_ - 1) / NT_;
+    const int sbeg = threadIdx.x * K;
+    int Lr[KMAX];
 #pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        const int head = g0 + g < G ? g0 + g : G - 1;
-        const float mk = ok ? __ldcg(p.part_ml + (slot * G + head) * 2) : -INFINITY;
-        const float lk = ok ? __ldcg(p.part_ml + (slot * G + head) * 2 + 1) : 0.f;
-        float cm = mk;
+    for (int k = 0; k < KMAX; ++k)
+      Lr[k] = (k < K && sbeg + k < S) ? __ldg(p.context_lens + sbeg + k) : 0;
+    int mine = 0;
 #pragma unroll
-        for (int x = 16; x > 0; x >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, x));
-        const float Mn = fmaxf(M[g], cm);
-        const float so = Mn == -INFINITY ? 0.f : exp2f(M[g] - Mn);
-        wk[g] = (mk == -INFINITY) ? 0.f : exp2f(mk - Mn);
-        float dl = wk[g] * lk;
-#pragma unroll
-        for (int x = 16; x > 0; x >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, x);
-        den[g] = den[g] * so + dl;
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) num[g][v] *= so;
-        M[g] = Mn;
-      }
-      for (int j0 = 0; j0 < cnt; j0 += UNR) {
-        VecT buf[UNR][GMAX];
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-          const int j = j0 + u < cnt ? j0 + u : cnt - 1;
-          const long long sj = __shfl_sync(0xffffffffu, slot, j);
-#pragma unroll
-          for (int g = 0; g < GMAX; ++g) {
-            const int head = g0 + g < G ? g0 + g : G - 1;
-            buf[u][g] = __ldcg(reinterpret_cast<const VecT *>(p.part_o + (sj * G + head) * D +
-                                                              lane * VPL));
-          }
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < K && sbeg + k < S) {
+        int L = Lr[k];
+        if (L < 0 || L > cap) {
+          if (zero_rows && blockIdx.x == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
+          L = L < 0 ? 0 : cap;
         }
+        Lr[k] = L;
+        mine += ceil_div_i(L, B);
+        if (L == 0 && ((sbeg + k) % gridDim.x) == blockIdx.x) zero_row(sbeg + k);
+      }
+    }
+    int incl = mine;
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-          const int j = j0 + u;
+    for (int x = 1; x < 32; x <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, x);
+      if (lane >= x) incl += v;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    long long before_warp = 0, tot = 0;
 #pragma unroll
-          for (int g = 0; g < GMAX; ++g) {
-            float wj = __shfl_sync(0xffffffffu, wk[g], j < cnt ? j : 0);
-            wj = j < cnt ? wj : 0.f;
-            num[g][0] = fmaf(wj, buf[u][g].x, num[g][0]);
-            num[g][1] = fmaf(wj, buf[u][g].y, num[g][1]);
-            if constexpr (VPL == 4) {
-              num[g][2] = fmaf(wj, reinterpret_cast<const float4 &>(buf[u][g]).z, num[g][2]);
-              num[g][3] = fmaf(wj, reinterpret_cast<const float4 &>(buf[u][g]).w, num[g][3]);
+    for (int k = 0; k < NW; ++k) {
+      if (k < warp) before_warp += red[k];
+      tot += red[k];
+    }
+    set_ranges(tot);
+    long long cum = before_warp + incl - mine;   // blocks before sequence sbeg
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < K && sbeg + k < S) {
+        const int nb = ceil_div_i(Lr[k], B);
+        if (nb > 0) {
+          const long long lo = cum * Hkv, hi = (cum + nb) * Hkv;
+          for (int kk = 0; kk < NW; ++kk) {
+            const long long uk = warp_u0(kk);
+            if (uk >= lo && uk < hi) {
+              loc_s[kk] = sbeg + k;
+              loc_base[kk] = lo;
+              loc_L[kk] = Lr[k];
             }
           }
         }
+        cum += nb;
       }
     }
+  } else {
+    // many sequences: a pass for the total, then a chunked scan
+    long long mine = 0;
+    for (int s = threadIdx.x; s < S; s += NT_) {
+      const int nb = seq_blocks<B>(p, s, zero_rows && blockIdx.x == 0);
+      mine += nb;
+      if (nb == 0 && (s % gridDim.x) == blockIdx.x) zero_row(s);
+    }
 #pragma unroll
-    for (int g = 0; g < GMAX; ++g) {
-      const int head = g0 + g;
-      if (head < G) {
-        const float inv = den[g] > 0.f ? 1.f / den[g] : 0.f;
-        if constexpr (VPL == 4) {
-          *reinterpret_cast<float4 *>(dst + head * D) =
-              make_float4(num[g][0] * inv, num[g][1] * inv, num[g][2] * inv, num[g][3] * inv);
-        } else {
-          *reinterpret_cast<float2 *>(dst + head * D) =
-              make_float2(num[g][0] * inv, num[g][1] * inv);
+    for (int x = 16; x > 0; x >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, x);
+    if (lane == 0) red[warp] = mine;
+    __syncthreads();
+    long long tot = 0;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) tot += red[k];
+    set_ranges(tot);
+    long long cta_max_u0 = -1;
+    for (int k = 0; k < NW; ++k) cta_max_u0 = max(cta_max_u0, warp_u0(k));
+    if (cta_max_u0 >= 0) {
+      long long run = 0;
+      for (int c0 = 0; c0 < S; c0 += NT_) {
+        const int s = c0 + threadIdx.x;
+        const int L = s < S ? seq_len_clamped<B>(p, s) : 0;
+        const int nb = ceil_div_i(L, B);
+        int incl = nb;
+#pragma unroll
+        for (int x = 1; x < 32; x <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, x);
+          if (lane >= x) incl += v;
         }
+        __syncthreads();
+        if (lane == 31) red[warp] = incl;
+        __syncthreads();
+        long long before_warp = 0, chunk_tot = 0;
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+          if (k < warp) before_warp += red[k];
+          chunk_tot += red[k];
+        }
+        const long long before = run + before_warp + incl - nb;   // blocks before seq s
+        if (nb > 0) {
+          const long long lo = before * Hkv, hi = (before + nb) * Hkv;
+          for (int kk = 0; kk < NW; ++kk) {
+            const long long uk = warp_u0(kk);
+            if (uk >= lo && uk < hi) {
+              loc_s[kk] = s;
+              loc_base[kk] = lo;
+              loc_L[kk] = L;
+            }
+          }
+        }
+        run += chunk_tot;
+        if (run * Hkv > cta_max_u0) break;
       }
     }
   }
+  __syncthreads();
 }
 
 // ============================================================================
@@ -679,142 +734,15 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   allow_dependent_launch();   // the split merge may be scheduled meanwhile
 
   // ---- plan: total tiles, this CTA's warp ranges ---------------------------
-  // Every CTA reads all context lengths once, scans their block counts, and
-  // finds the sequence holding the first tile of each of its warps.
-  constexpr int NT_ = NW * 32;   // threads per CTA
-  constexpr int KMAX = 8;   // sequences per thread on the one-pass path
   const long long w_total = (long long)gridDim.x * NW;
   const long long w = (long long)blockIdx.x * NW + warp;
   long long U = 0, w_active = 0;
-  auto set_ranges = [&](long long tot) {
-    U = tot * Hkv;
-    w_active = 0;
-    if (U > 0) {
-      w_active = (U + p.min_tiles - 1) / p.min_tiles;
-      if (w_active > w_total) w_active = w_total;
-    }
-  };
-  auto warp_u0 = [&](int k) -> long long {   // first tile of this CTA's warp k, -1 if idle
-    const long long wk = (long long)blockIdx.x * NW + k;
-    return wk < w_active ? (wk * U) / w_active : -1;
-  };
-  auto zero_row = [&](int s) {   // empty sequence: zero output rows
-    float4 *row = reinterpret_cast<float4 *>(p.out + (int64_t)s * p.num_q_heads * D);
-    for (int k = 0; k < p.num_q_heads * D / 4; ++k) row[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  };
-  const int cap = p.max_blocks * B;
-  if (S <= NT_ * KMAX) {
-    // one pass: thread t owns sequences [t*K, t*K + K)
-    const int K = (S + NT_ - 1) / NT_;
-    const int sbeg = threadIdx.x * K;
-    int Lr[KMAX];
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k)
-      Lr[k] = (k < K && sbeg + k < S) ? __ldg(p.context_lens + sbeg + k) : 0;
-    int mine = 0;
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-      if (k < K && sbeg + k < S) {
-        int L = Lr[k];
-        if (L < 0 || L > cap) {
-          if (blockIdx.x == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
-          L = L < 0 ? 0 : cap;
-        }
-        Lr[k] = L;
-        mine += ceil_div_i(L, B);
-        if (L == 0 && ((sbeg + k) % gridDim.x) == blockIdx.x) zero_row(sbeg + k);
-      }
-    }
-    int incl = mine;
-#pragma unroll
-    for (int x = 1; x < 32; x <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, x);
-      if (lane >= x) incl += v;
-    }
-    if (lane == 31) red[warp] = incl;
-    __syncthreads();
-    long long before_warp = 0, tot = 0;
-#pragma unroll
-    for (int k = 0; k < NW; ++k) {
-      if (k < warp) before_warp += red[k];
-      tot += red[k];
-    }
-    set_ranges(tot);
-    long long cum = before_warp + incl - mine;   // blocks before sequence sbeg
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-      if (k < K && sbeg + k < S) {
-        const int nb = ceil_div_i(Lr[k], B);
-        if (nb > 0) {
-          const long long lo = cum * Hkv, hi = (cum + nb) * Hkv;
-          for (int kk = 0; kk < NW; ++kk) {
-            const long long uk = warp_u0(kk);
-            if (uk >= lo && uk < hi) {
-              loc_s[kk] = sbeg + k;
-              loc_base[kk] = lo;
-              loc_L[kk] = Lr[k];
-            }
-          }
-        }
-        cum += nb;
-      }
-    }
-  } else {
-    // many sequences: a pass for the total, then a chunked scan
-    long long mine = 0;
-    for (int s = threadIdx.x; s < S; s += NT_) {
-      const int nb = seq_blocks<B>(p, s, blockIdx.x == 0);
-      mine += nb;
-      if (nb == 0 && (s % gridDim.x) == blockIdx.x) zero_row(s);
-    }
-#pragma unroll
-    for (int x = 16; x > 0; x >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, x);
-    if (lane == 0) red[warp] = mine;
-    __syncthreads();
-    long long tot = 0;
-#pragma unroll
-    for (int k = 0; k < NW; ++k) tot += red[k];
-    set_ranges(tot);
-    long long cta_max_u0 = -1;
-    for (int k = 0; k < NW; ++k) cta_max_u0 = max(cta_max_u0, warp_u0(k));
-    if (cta_max_u0 >= 0) {
-      long long run = 0;
-      for (int c0 = 0; c0 < S; c0 += NT_) {
-        const int s = c0 + threadIdx.x;
-        const int L = s < S ? seq_len_clamped<B>(p, s) : 0;
-        const int nb = ceil_div_i(L, B);
-        int incl = nb;
-#pragma unroll
-        for (int x = 1; x < 32; x <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, x);
-          if (lane >= x) incl += v;
-        }
-        __syncthreads();
-        if (lane == 31) red[warp] = incl;
-        __syncthreads();
-        long long before_warp = 0, chunk_tot = 0;
-#pragma unroll
-        for (int k = 0; k < NW; ++k) {
-          if (k < warp) before_warp += red[k];
-          chunk_tot += red[k];
-        }
-        const long long before = run + before_warp + incl - nb;   // blocks before seq s
-        if (nb > 0) {
-          const long long lo = before * Hkv, hi = (before + nb) * Hkv;
-          for (int kk = 0; kk < NW; ++kk) {
-            const long long uk = warp_u0(kk);
-            if (uk >= lo && uk < hi) {
-              loc_s[kk] = s;
-              loc_base[kk] = lo;
-              loc_L[kk] = L;
-            }
-          }
-        }
-        run += chunk_tot;
-        if (run * Hkv > cta_max_u0) break;
-      }
-    }
-  }
+  cta_plan<B, NW>(
+      p, w_total, [&](int k, long long U_, long long wa_) -> long long {
+        const long long wk = (long long)blockIdx.x * NW + k;   // first tile of warp k
+        return wk < wa_ ? (wk * U_) / wa_ : -1;
+      },
+      true, red, loc_s, loc_base, loc_L, U, w_active);
   __syncthreads();
   if (lane == 0) fence_barrier_init();
   __syncwarp();
@@ -834,10 +762,20 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   const long long r0 = u0 - base0;
   const int h0 = (int)(r0 / nb0);
   const int j0 = (int)(r0 - (long long)h0 * nb0);
-  if (lane < kMetaWords) {
+  if (lane < kMetaWords) {   // descriptor: u0, first segment [lo, hi), U, active warps, s, h
     const long long seg_lo = base0 + (long long)h0 * nb0;
-    const long long v[kMetaWords] = {u0, seg_lo, seg_lo + nb0, U, w_active, s0, h0, 1};
-    meta[lane] = v[lane];
+    long long v = 1;
+    switch (lane) {
+      case 0: v = u0; break;
+      case 1: v = seg_lo; break;
+      case 2: v = seg_lo + nb0; break;
+      case 3: v = U; break;
+      case 4: v = w_active; break;
+      case 5: v = s0; break;
+      case 6: v = h0; break;
+      default: v = 1;
+    }
+    meta[lane] = v;
   }
   const long long ntiles = u1 - u0;
 
@@ -993,20 +931,28 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
 }
 
 // ============================================================================
-// Merge of split segments: one warp per boundary b between warp ranges b-1
-// and b; the warp merges the segment the boundary cuts if it is the first
-// boundary inside that segment.  Launched as a programmatic dependent of the
-// streaming kernel.
+// Merge of split segments.  Warp t of the grid handles boundary b = t / hc + 1
+// between warp ranges b-1 and b, and heads [c*GMW, (c+1)*GMW) of the group,
+// c = t % hc: if b is the first boundary inside the segment it cuts, the warp
+// merges those heads' partials (several warps share a segment with many
+// heads, so long segments with many partials are merged in parallel).
+// Launched as a programmatic dependent of the streaming kernel.
 // ============================================================================
-template <int D, int GMAX>
-__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p, int w_total) {
+template <int D, int GMW>
+__global__ void __launch_bounds__(128, 6)
+    paged_decode_merge_kernel(const DecodeParams p, int w_total, int hc) {
+  constexpr int VPL = D / 32;
+  constexpr int UNR = 8 / GMW;   // partials per batch of loads
+  using VecT = typename std::conditional<VPL == 4, float4, float2>::type;
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
-  const long long b = (long long)blockIdx.x * 4 + (threadIdx.x >> 5) + 1;
+  const long long t = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const long long b = t / hc + 1;
+  const int c = (int)(t % hc);
   if (b >= w_total) return;
   const long long mv = lane < kMetaWords ? __ldcg(p.meta + b * kMetaWords + lane)
                                          : __ldcg(p.meta + (b - 1) * kMetaWords);
-  const long long u0b = __shfl_sync(0xffffffffu, mv, 0);
+  const long long ub = __shfl_sync(0xffffffffu, mv, 0);
   const long long lo = __shfl_sync(0xffffffffu, mv, 1);
   const long long hi = __shfl_sync(0xffffffffu, mv, 2);
   const long long U = __shfl_sync(0xffffffffu, mv, 3);
@@ -1014,9 +960,92 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
   const int s = (int)__shfl_sync(0xffffffffu, mv, 5);
   const int h = (int)__shfl_sync(0xffffffffu, mv, 6);
   const long long active = __shfl_sync(0xffffffffu, mv, 7);
-  const long long u0a = __shfl_sync(0xffffffffu, mv, 8);
-  if (!active || lo >= u0b || lo < u0a) return;
-  merge_parts<D, GMAX>(p, s, h, lo, hi, U, wa, lane);
+  const long long uprev = __shfl_sync(0xffffffffu, mv, 8);
+  // merge only at the first boundary inside a cut segment
+  if (!active || lo >= ub || lo < uprev) return;
+  const int G = p.group;
+  const int g0 = c * GMW;
+  if (g0 >= G) return;
+
+  const long long c_lo = warp_of(lo, U, wa), c_hi = warp_of(hi - 1, U, wa);
+  const long long n = c_hi - c_lo + 1;
+  float M[GMW], den[GMW], num[GMW][VPL];
+#pragma unroll
+  for (int g = 0; g < GMW; ++g) {
+    M[g] = -INFINITY;
+    den[g] = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) num[g][v] = 0.f;
+  }
+  for (long long k0 = 0; k0 < n; k0 += 32) {
+    const long long k = k0 + lane;
+    const bool ok = k < n;
+    const long long slot = ok ? part_slot(c_lo + k, lo, U, wa) : 0;
+    const int cnt = (int)((n - k0) < 32 ? (n - k0) : 32);
+    float wk[GMW];
+#pragma unroll
+    for (int g = 0; g < GMW; ++g) {
+      const int head = g0 + g < G ? g0 + g : G - 1;
+      const float mk = ok ? __ldcg(p.part_ml + (slot * G + head) * 2) : -INFINITY;
+      const float lk = ok ? __ldcg(p.part_ml + (slot * G + head) * 2 + 1) : 0.f;
+      float cm = mk;
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, x));
+      const float Mn = fmaxf(M[g], cm);
+      const float so = Mn == -INFINITY ? 0.f : exp2f(M[g] - Mn);
+      wk[g] = (mk == -INFINITY) ? 0.f : exp2f(mk - Mn);
+      float dl = wk[g] * lk;
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, x);
+      den[g] = den[g] * so + dl;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) num[g][v] *= so;
+      M[g] = Mn;
+    }
+    for (int j0 = 0; j0 < cnt; j0 += UNR) {
+      VecT buf[UNR][GMW];
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        const int j = j0 + u < cnt ? j0 + u : cnt - 1;
+        const long long sj = __shfl_sync(0xffffffffu, slot, j);
+#pragma unroll
+        for (int g = 0; g < GMW; ++g) {
+          const int head = g0 + g < G ? g0 + g : G - 1;
+          buf[u][g] = __ldcg(reinterpret_cast<const VecT *>(p.part_o + (sj * G + head) * D +
+                                                            lane * VPL));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        const int j = j0 + u;
+#pragma unroll
+        for (int g = 0; g < GMW; ++g) {
+          float wj = __shfl_sync(0xffffffffu, wk[g], j < cnt ? j : 0);
+          wj = j < cnt ? wj : 0.f;
+          num[g][0] = fmaf(wj, buf[u][g].x, num[g][0]);
+          num[g][1] = fmaf(wj, buf[u][g].y, num[g][1]);
+          if constexpr (VPL == 4) {
+            num[g][2] = fmaf(wj, reinterpret_cast<const float4 &>(buf[u][g]).z, num[g][2]);
+            num[g][3] = fmaf(wj, reinterpret_cast<const float4 &>(buf[u][g]).w, num[g][3]);
+          }
+        }
+      }
+    }
+  }
+  float *dst = p.out + ((int64_t)s * p.num_q_heads + (int64_t)h * G) * D + lane * VPL;
+#pragma unroll
+  for (int g = 0; g < GMW; ++g) {
+    const int head = g0 + g;
+    if (head < G) {
+      const float inv = den[g] > 0.f ? 1.f / den[g] : 0.f;
+      if constexpr (VPL == 4) {
+        *reinterpret_cast<float4 *>(dst + head * D) =
+            make_float4(num[g][0] * inv, num[g][1] * inv, num[g][2] * inv, num[g][3] * inv);
+      } else {
+        *reinterpret_cast<float2 *>(dst + head * D) = make_float2(num[g][0] * inv, num[g][1] * inv);
+      }
+    }
+  }
 }
 
 }  // namespace pa

@@ -195,6 +195,7 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   p.num_q_heads = a.num_q_heads;
   p.num_kv_heads = a.num_kv_heads;
   p.group = G;
+  p.head_dim = D;
   p.max_blocks = a.max_blocks;
   p.num_blocks = a.num_blocks;
   p.nstage = L.nstage;
@@ -218,19 +219,26 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
     cudaGetLastError();
     return PA_ERR_CUDA;
   }
-  // Split merge: one warp per boundary between warp ranges, scheduled as the
-  // streaming CTAs retire and released when the streaming grid completes.
+  // Split merge: one warp per (boundary between warp ranges, group of up to
+  // four heads, two when the group is larger), resident and waiting before
+  // the streaming grid completes.
   if (L.w_total > 1) {
-    constexpr int GMAX = NT == 0 ? 1 : 4;
     cudaLaunchConfig_t mc = {};
-    mc.gridDim = dim3((unsigned)((L.w_total - 1 + 3) / 4));
     mc.blockDim = dim3(128);
     mc.dynamicSmemBytes = 0;
     mc.stream = a.stream;
     mc.attrs = attr;
     mc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&mc, pa::paged_decode_merge_kernel<D, GMAX>, p, L.w_total) !=
-        cudaSuccess) {
+    cudaError_t e;
+    if (G <= 4) {
+      mc.gridDim = dim3((unsigned)((L.w_total - 1 + 3) / 4));
+      e = cudaLaunchKernelEx(&mc, pa::paged_decode_merge_kernel<D, 4>, p, L.w_total, 1);
+    } else {
+      const int hc = (G + 1) / 2;
+      mc.gridDim = dim3((unsigned)(((long long)(L.w_total - 1) * hc + 3) / 4));
+      e = cudaLaunchKernelEx(&mc, pa::paged_decode_merge_kernel<D, 2>, p, L.w_total, hc);
+    }
+    if (e != cudaSuccess) {
       cudaGetLastError();
       return PA_ERR_CUDA;
     }
@@ -481,8 +489,8 @@ int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_
   void *scratch = nullptr;
   const int st = no_alloc_scratch(dev, &scratch);
   if (st != PA_OK) return st;
-  // The scratch needs no clearing: every descriptor and partial the merge
-  // reads is written by the same call's streaming kernel first.  A launch that needs more than
+  // The scratch needs no clearing: every partial the merge reads is written
+  // by the same call's streaming kernel first.  A launch that needs more than
   // kNoAllocScratchBytes is refused by launch_decode with PA_ERR_WORKSPACE.
   DecodeArgs a{out,          q,           k_cache,      v_cache,      nullptr,
                nullptr,      block_tables, context_lens, scale,        num_kv_heads,
