@@ -296,6 +296,22 @@ int pa_bm_ref_count(const pa_bm *bm, int32_t block);
 /* Number of live sequences. */
 int pa_bm_num_seqs(const pa_bm *bm);
 
+/*
+ * KV memory accounting of the pool ([P1] section 1 "The Contiguous
+ * Allocation Problem" and section 3: paged blocks leave idle only the tail of
+ * each sequence's last block, and shared prompt blocks are stored once).
+ *   used_blocks    distinct blocks held by some sequence
+ *   shared_blocks  blocks held by more than one sequence
+ *   logical_tokens sum of the sequences' lengths (shared tokens counted per holder)
+ *   filled_slots   sum over used blocks of the largest fill any holder gives it
+ * The idle slots are used_blocks * block_size - filled_slots.
+ */
+typedef struct {
+  int64_t num_blocks, free_blocks, used_blocks, shared_blocks;
+  int64_t num_seqs, logical_tokens, filled_slots, block_size;
+} pa_bm_stats_t;
+int pa_bm_stats(const pa_bm *bm, pa_bm_stats_t *out);
+
 #ifdef __cplusplus
 }
 #endif

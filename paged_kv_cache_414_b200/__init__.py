@@ -57,6 +57,12 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+class BmStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("num_blocks", "free_blocks", "used_blocks",
+                                               "shared_blocks", "num_seqs", "logical_tokens",
+                                               "filled_slots", "block_size")]
+
+
 def _declare(L):
     c = ctypes
     vp, i32, i64, sz, f32 = c.c_void_p, c.c_int, c.c_int64, c.c_size_t, c.c_float
@@ -88,6 +94,7 @@ def _declare(L):
         "pa_bm_num_free": (i32, [vp]),
         "pa_bm_ref_count": (i32, [vp, c.c_int32]),
         "pa_bm_num_seqs": (i32, [vp]),
+        "pa_bm_stats": (i32, [vp, c.POINTER(BmStats)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -393,6 +400,35 @@ class BlockManager:
 
     def num_seqs(self) -> int:
         return lib().pa_bm_num_seqs(self._h)
+
+    def stats(self) -> dict:
+        """pa_bm_stats: blocks used / shared / free, tokens, filled slots, plus
+        the derived idle slots and waste fraction."""
+        st = BmStats()
+        _check(lib().pa_bm_stats(self._h, ctypes.byref(st)), "pa_bm_stats")
+        d = {name: int(getattr(st, name)) for name, _ in BmStats._fields_}
+        slots = d["used_blocks"] * d["block_size"]
+        d["idle_slots"] = slots - d["filled_slots"]
+        d["waste_fraction"] = d["idle_slots"] / slots if slots else 0.0
+        return d
+
+
+def utilisation_report(bm: "BlockManager", reserve: int) -> dict:
+    """Paged KV memory of the manager's live sequences against a contiguous
+    reservation of `reserve` tokens per sequence (the allocation PagedAttention
+    replaces): slots allocated, useful fraction, idle slots, for both."""
+    st = bm.stats()
+    contiguous = st["num_seqs"] * reserve
+    paged = st["used_blocks"] * st["block_size"]
+    return {
+        "paged_slots": paged,
+        "paged_useful_fraction": st["filled_slots"] / paged if paged else 1.0,
+        "paged_idle_slots": st["idle_slots"],
+        "contiguous_slots": contiguous,
+        "contiguous_useful_fraction": st["logical_tokens"] / contiguous if contiguous else 1.0,
+        "contiguous_idle_slots": contiguous - st["logical_tokens"],
+        "sharing_ratio": st["logical_tokens"] / st["filled_slots"] if st["filled_slots"] else 1.0,
+    }
 
 
 def decode_bytes(context_lens, num_kv_heads: int, head_dim: int, block_size: int,

@@ -255,4 +255,34 @@ int pa_bm_ref_count(const pa_bm *bm, int32_t block) {
 
 int pa_bm_num_seqs(const pa_bm *bm) { return bm ? (int)bm->seqs.size() : PA_ERR_ARG; }
 
+int pa_bm_stats(const pa_bm *bm, pa_bm_stats_t *out) {
+  if (!bm || !out) return PA_ERR_ARG;
+  // filled slots of each block in use: the largest fill any holder gives it
+  std::unordered_map<int32_t, int> fill;
+  int64_t logical = 0;
+  for (const auto &kv : bm->seqs) {
+    const Seq &s = kv.second;
+    logical += s.len;
+    for (size_t j = 0; j < s.table.size(); ++j) {
+      const int64_t n = std::min<int64_t>(bm->block_size, s.len - (int64_t)j * bm->block_size);
+      int &f = fill[s.table[j]];
+      f = std::max<int>(f, (int)n);
+    }
+  }
+  int64_t filled = 0, shared = 0;
+  for (const auto &kv : fill) {
+    filled += kv.second;
+    if (bm->ref[kv.first] > 1) ++shared;
+  }
+  out->num_blocks = bm->num_blocks;
+  out->free_blocks = (int64_t)bm->free_list.size();
+  out->used_blocks = (int64_t)fill.size();
+  out->shared_blocks = shared;
+  out->num_seqs = (int64_t)bm->seqs.size();
+  out->logical_tokens = logical;
+  out->filled_slots = filled;
+  out->block_size = bm->block_size;
+  return PA_OK;
+}
+
 }  // extern "C"

@@ -809,6 +809,9 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   nxt = follow(cur, ntiles - cur.n);
 
   const uint8_t *qbase = p.q;
+  // K/V tiles are read once per call: evict them from L2 first, so the
+  // partials this call writes for the split merge are still there for it.
+  const uint64_t stream_policy = l2_policy_evict_first();
   auto issue = [&](int stage) {
     if (cur_k == cur.n) {
       cur = nxt;
@@ -849,8 +852,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
           uint8_t *kd = stages + (size_t)stage * STAGE;
 #pragma unroll
           for (int bx = 0; bx < D / 64; ++bx) {
-            tma_load_2d(kd + bx * (B * 128), &kmap, bx * 64, row, bar);
-            tma_load_2d(kd + TILE + bx * (B * 128), &vmap, bx * 64, row, bar);
+            tma_load_2d_hint(kd + bx * (B * 128), &kmap, bx * 64, row, bar, stream_policy);
+            tma_load_2d_hint(kd + TILE + bx * (B * 128), &vmap, bx * 64, row, bar, stream_policy);
           }
         }
         if (flags & TF_FIRST)
