@@ -143,7 +143,7 @@ def test_device_checks_report_instead_of_faulting(pa, cuda_device):
     out = torch.empty(2, 4, 64, device=dev)
     pa.pa_paged_decode_attention(out, b.q, b.k_cache, b.v_cache, tables, lens, b.scale, 2)
     assert pa.pa_device_error() & pa.DEVERR["block_id"]
-    lens2 = lens.clone(); lens2[0] = 10_000
+    lens2 = torch.as_tensor(np.array([10_000, 40], dtype=np.int32), device=dev)
     pa.pa_paged_decode_attention(out, b.q, b.k_cache, b.v_cache,
                                  torch.as_tensor(b.block_tables, device=dev), lens2, b.scale, 2,
                                  max_context_len=b.max_blocks_per_seq * 16)
