@@ -55,7 +55,7 @@ KERNEL_SOURCES = ["paged_kv_cache_414_b200/csrc/decode_attention.cuh",
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa8b", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
@@ -390,11 +390,13 @@ def run_b200(args, rank, world, local_rank):
 
 def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
     """Same metric through the public API from pinned host buffers: per step,
-    the host block manager reserves the slots, the step's inputs (q, new K/V,
-    slots, block tables, lengths) go host -> device, the library's kernels
-    run, and the output comes back device -> host.  Three streams (upload,
-    compute, download) and three buffer sets let step i+1's upload and step
-    i-1's download overlap step i's kernels; events order every reuse."""
+    the host block manager reserves the slots and writes the block tables
+    straight into pinned memory, the step's inputs (q, new K/V, lengths,
+    block tables, copy-on-write pairs) go host -> device as one packed copy,
+    the library's kernels run, and the output comes back device -> host.
+    Three streams (upload, compute, download) and three buffer sets let step
+    i+1's upload and step i-1's download overlap step i's kernels; events
+    order every reuse."""
     import torch
     import torch.distributed as dist
     sh = wl.shape
@@ -403,75 +405,86 @@ def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
     seqs = np.arange(S)
     bm = wl.new_manager(pa)
     NBUF = 3
-    h_q = [b.q.cpu().pin_memory() for _ in range(NBUF)]
-    h_k = [b.k_new.cpu().pin_memory() for _ in range(NBUF)]
-    h_v = [b.v_new.cpu().pin_memory() for _ in range(NBUF)]
-    h_slots = [torch.empty(S, dtype=torch.int64).pin_memory() for _ in range(NBUF)]
-    h_tables = [torch.empty(S, wl.maxb, dtype=torch.int32).pin_memory() for _ in range(NBUF)]
-    h_lens = [torch.empty(S, dtype=torch.int32).pin_memory() for _ in range(NBUF)]
+
+    # packed input layout: q | k_new | v_new | lens | tables | pairs (256-byte aligned)
+    def al(n):
+        return (n + 255) // 256 * 256
+    parts = [("q", b.q.dtype, (S, sh.num_q_heads, sh.head_dim), 2),
+             ("k", b.k_new.dtype, (S, sh.num_kv_heads, sh.head_dim), 2),
+             ("v", b.v_new.dtype, (S, sh.num_kv_heads, sh.head_dim), 2),
+             ("lens", torch.int32, (S,), 4),
+             ("tables", torch.int32, (S, wl.maxb), 4),
+             ("pairs", torch.int64, (S, 2), 8)]
+    off, pos = {}, 0
+    for name, _, shape, es in parts:
+        off[name] = pos
+        pos += al(int(np.prod(shape)) * es)
+    total = pos
+
+    def views(buf):
+        v = {}
+        for name, dt, shape, es in parts:
+            n = int(np.prod(shape)) * es
+            v[name] = buf[off[name]:off[name] + n].view(dt).view(shape)
+        return v
+
+    h_buf = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(NBUF)]
+    d_buf = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(NBUF)]
+    h_in = [views(x) for x in h_buf]
+    d_in = [views(x) for x in d_buf]
+    h_slots = [np.empty(S, dtype=np.int64) for _ in range(NBUF)]
+    for hv in h_in:
+        hv["q"].copy_(b.q.cpu())
+        hv["k"].copy_(b.k_new.cpu())
+        hv["v"].copy_(b.v_new.cpu())
     h_out = [torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32).pin_memory()
              for _ in range(NBUF)]
-    d_q = [torch.empty_like(b.q) for _ in range(NBUF)]
-    d_k = [torch.empty_like(b.k_new) for _ in range(NBUF)]
-    d_v = [torch.empty_like(b.v_new) for _ in range(NBUF)]
-    d_slots = [torch.empty(S, dtype=torch.int64, device=dev) for _ in range(NBUF)]
-    d_tables = [torch.empty(S, wl.maxb, dtype=torch.int32, device=dev) for _ in range(NBUF)]
-    d_lens = [torch.empty(S, dtype=torch.int32, device=dev) for _ in range(NBUF)]
-    d_pairs = [torch.empty(S, 2, dtype=torch.int64, device=dev) for _ in range(NBUF)]
-    h_pairs = [torch.empty(S, 2, dtype=torch.int64).pin_memory() for _ in range(NBUF)]
     d_out = [torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
              for _ in range(NBUF)]
     maxctx = wl.maxb * B
     ws = pa.alloc_workspace(S, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, B, maxctx, dev)
     s_up, s_cmp, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_up = [None] * NBUF    # upload of the set done
-    ev_cmp = [None] * NBUF   # kernels that read the set's inputs / write its output done
-    ev_dn = [None] * NBUF    # download of the set's output done
-    h2d = sum(t[0].numel() * t[0].element_size() for t in (h_q, h_k, h_v, h_tables, h_lens))
-    d2h = h_out[0].numel() * 4
+    ev_up = [torch.cuda.Event() for _ in range(NBUF)]    # upload of the set done
+    ev_cmp = [torch.cuda.Event() for _ in range(NBUF)]   # kernels reading / writing the set done
+    ev_dn = [torch.cuda.Event() for _ in range(NBUF)]    # download of the set's output done
+    used = [False] * NBUF
+    in_bytes = off["pairs"]                      # everything up to the (optional) pairs
+    h2d_steps, d2h = [], h_out[0].numel() * 4
 
     def one(i):
         j = i % NBUF
-        if ev_up[j] is not None:
+        hv, dv = h_in[j], d_in[j]
+        if used[j]:
             ev_up[j].synchronize()             # host buffers of set j are free again
-        slots, pairs = bm.append_slots(seqs)
-        h_slots[j].numpy()[:] = slots
-        tables, lens = bm.block_tables(seqs, wl.maxb)
-        h_tables[j].numpy()[:] = tables
-        h_lens[j].numpy()[:] = lens
+        _, pairs = bm.append_slots(seqs, slots_out=h_slots[j], pairs_out=hv["pairs"])
+        bm.block_tables(seqs, wl.maxb, out=hv["tables"], lens_out=hv["lens"])
         npairs = len(pairs)
-        if npairs:
-            h_pairs[j].numpy()[:npairs] = pairs
+        nbytes = in_bytes + npairs * 16
+        h2d_steps.append(nbytes)
         with torch.cuda.stream(s_up):
-            if ev_cmp[j] is not None:
+            if used[j]:
                 s_up.wait_event(ev_cmp[j])     # device inputs of set j no longer read
-            for d, h in ((d_q[j], h_q[j]), (d_k[j], h_k[j]), (d_v[j], h_v[j]),
-                         (d_tables[j], h_tables[j]), (d_lens[j], h_lens[j])):
-                d.copy_(h, non_blocking=True)
-            if npairs:
-                d_pairs[j][:npairs].copy_(h_pairs[j][:npairs], non_blocking=True)
-            ev_up[j] = torch.cuda.Event()
+            d_buf[j][:nbytes].copy_(h_buf[j][:nbytes], non_blocking=True)
             ev_up[j].record(s_up)
-        with torch.cuda.stream(s_cmp):
-            s_cmp.wait_event(ev_up[j])
-            if ev_dn[j] is not None:
-                s_cmp.wait_event(ev_dn[j])     # output of set j downloaded
-            if npairs:
-                pa.pa_copy_blocks(b.k_cache, b.v_cache, d_pairs[j][:npairs])
-            pa.pa_decode_step(d_out[j], d_q[j], d_k[j], d_v[j], b.k_cache, b.v_cache,
-                              d_tables[j], d_lens[j], wl.scale, sh.num_kv_heads,
-                              max_context_len=maxctx, workspace=ws)
-            ev_cmp[j] = torch.cuda.Event()
-            ev_cmp[j].record(s_cmp)
+        s_cmp.wait_event(ev_up[j])
+        if used[j]:
+            s_cmp.wait_event(ev_dn[j])         # output of set j downloaded
+        if npairs:
+            pa.pa_copy_blocks(b.k_cache, b.v_cache, dv["pairs"][:npairs], stream=s_cmp)
+        pa.pa_decode_step(d_out[j], dv["q"], dv["k"], dv["v"], b.k_cache, b.v_cache,
+                          dv["tables"], dv["lens"], wl.scale, sh.num_kv_heads,
+                          max_context_len=maxctx, workspace=ws, stream=s_cmp)
+        ev_cmp[j].record(s_cmp)
         with torch.cuda.stream(s_dn):
             s_dn.wait_event(ev_cmp[j])
             h_out[j].copy_(d_out[j], non_blocking=True)
-            ev_dn[j] = torch.cuda.Event()
             ev_dn[j].record(s_dn)
+        used[j] = True
 
     for i in range(Wm):
         one(i)
     torch.cuda.synchronize()
+    h2d_steps.clear()
     if world > 1:
         dist.barrier()
     t0 = time.perf_counter()
@@ -483,10 +496,12 @@ def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
     dt_max = reduce_max(dt)
     bytes_all = reduce_sum(float(sum(wl.bytes_per_step(i) for i in range(Wm, Wm + K))))
     return {"value": round(bytes_all / dt_max / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "h2d_bytes_per_step": int(round(sum(h2d_steps) / max(len(h2d_steps), 1))),
+            "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(dt_max * 1e3 / K, 4),
             "timing": "host wall clock, synchronize on both sides, max over ranks; "
-                      "upload / compute / download on three streams, three buffer sets"}
+                      "upload (one packed copy) / compute / download on three streams, "
+                      "three buffer sets"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)

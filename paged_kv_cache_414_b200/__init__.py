@@ -296,6 +296,17 @@ def pa_device_error(clear: bool = True) -> int:
 
 # --------------------------------------------------------------------------- block manager
 
+def _out(a, shape, dtype):
+    """A caller-provided output array (numpy, or a CPU torch tensor such as a
+    pinned buffer) checked for shape, dtype and contiguity."""
+    if not isinstance(a, np.ndarray):
+        a = a.numpy()
+    if a.shape != tuple(shape) or a.dtype != dtype or not a.flags.c_contiguous:
+        raise ValueError(f"output array must be contiguous {np.dtype(dtype)} {tuple(shape)}, "
+                         f"got {a.dtype} {a.shape}")
+    return a
+
+
 def _p64(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
 
@@ -350,16 +361,21 @@ class BlockManager:
             _check(r, "pa_bm_append_slot")
         return int(slot.value), ((int(cs.value), int(cd.value)) if r == 1 else None)
 
-    def append_slots(self, seqs):
-        """(slots int64 [n], cow_pairs int64 [k, 2]) for one append per entry."""
+    def append_slots(self, seqs, slots_out=None, pairs_out=None):
+        """(slots int64 [n], cow_pairs int64 [k, 2]) for one append per entry.
+        With `slots_out` ([n] int64) and `pairs_out` ([n, 2] int64), e.g. views
+        of pinned host memory, the results are written there and views of them
+        returned."""
         seqs = np.ascontiguousarray(seqs, dtype=np.int64)
         n = seqs.shape[0]
-        slots = np.empty(n, dtype=np.int64)
-        pairs = np.empty((max(n, 1), 2), dtype=np.int64)
+        slots = (np.empty(n, dtype=np.int64) if slots_out is None
+                 else _out(slots_out, (n,), np.int64))
+        pairs = (np.empty((max(n, 1), 2), dtype=np.int64) if pairs_out is None
+                 else _out(pairs_out, (max(n, 1), 2), np.int64))
         k = ctypes.c_int(0)
         _check(lib().pa_bm_append_slots(self._h, _p64(seqs), n, _p64(slots), _p64(pairs),
                                         ctypes.byref(k)), "pa_bm_append_slots")
-        return slots, pairs[:k.value].copy()
+        return slots, (pairs[:k.value] if pairs_out is not None else pairs[:k.value].copy())
 
     def free_seq(self, seq: int) -> None:
         _check(lib().pa_bm_free(self._h, seq), "pa_bm_free")
@@ -373,12 +389,13 @@ class BlockManager:
                "pa_bm_block_table")
         return out[:got.value].tolist()
 
-    def block_tables(self, seqs, cap: int):
-        """(tables int32 [n, cap] padded with -1, lens int32 [n])."""
+    def block_tables(self, seqs, cap: int, out=None, lens_out=None):
+        """(tables int32 [n, cap] padded with -1, lens int32 [n]); written into
+        `out` / `lens_out` when given (contiguous int32 arrays of those shapes)."""
         seqs = np.ascontiguousarray(seqs, dtype=np.int64)
         n = seqs.shape[0]
-        out = np.empty((n, cap), dtype=np.int32)
-        lens = np.empty(n, dtype=np.int32)
+        out = np.empty((n, cap), dtype=np.int32) if out is None else _out(out, (n, cap), np.int32)
+        lens = np.empty(n, dtype=np.int32) if lens_out is None else _out(lens_out, (n,), np.int32)
         _check(lib().pa_bm_block_tables(self._h, _p64(seqs), n, _p32(out), cap, _p32(lens)),
                "pa_bm_block_tables")
         return out, lens

@@ -147,3 +147,40 @@ def test_native_errors_leave_state_unchanged(pa):
                       nat.seq_len(1))
     with pytest.raises(ValueError):
         pa.BlockManager(4, 4, [0, 1, 1, 2])
+
+
+def test_outputs_into_caller_buffers(pa):
+    """append_slots / block_tables write into caller arrays (numpy or a CPU
+    torch tensor, as a pinned upload buffer would be) exactly what they
+    return otherwise; a wrong shape or dtype is refused."""
+    import torch
+    wl = W.cow_workload(steps=4)
+    B = wl.shape.block_size
+    mk = []
+    for _ in range(2):
+        bm = pa.BlockManager(wl.num_blocks, B, wl.free_order)
+        for p, P in enumerate(wl.prompt_lens):
+            bm.allocate(wl.seq_id(p, 0), int(P))
+            for br in range(1, wl.branches):
+                bm.fork(wl.seq_id(p, 0), wl.seq_id(p, br))
+        mk.append(bm)
+    a, b = mk
+    seqs = np.arange(wl.num_seqs)
+    n = len(seqs)
+    slots_buf = np.full(n, -7, dtype=np.int64)
+    pairs_buf = torch.full((n, 2), -7, dtype=torch.int64)
+    tab_buf = torch.full((n, 64), -7, dtype=torch.int32)
+    lens_buf = np.full(n, -7, dtype=np.int32)
+    for _ in range(wl.steps):
+        s1, p1 = a.append_slots(seqs)
+        s2, p2 = b.append_slots(seqs, slots_out=slots_buf, pairs_out=pairs_buf)
+        assert np.array_equal(s1, s2) and np.array_equal(s1, slots_buf)
+        assert np.array_equal(p1, p2) and np.array_equal(p1, pairs_buf.numpy()[:len(p1)])
+        t1, l1 = a.block_tables(seqs, 64)
+        b.block_tables(seqs, 64, out=tab_buf, lens_out=lens_buf)
+        assert np.array_equal(t1, tab_buf.numpy()) and np.array_equal(l1, lens_buf)
+    with pytest.raises(ValueError):
+        b.block_tables(seqs, 64, out=np.empty((n, 63), dtype=np.int32))
+    with pytest.raises(ValueError):
+        b.append_slots(seqs, slots_out=np.empty(n, dtype=np.int32))
+    a.close(); b.close()
