@@ -14,7 +14,8 @@ Everything is written to be checked by eye against the pages it follows:
                     partial/merge algebra.
 * ``cache_ops``     reshape_and_cache (scatter of new K/V into their slots) and
                     copy_blocks (copy-on-write block copies), on raw bits.
-* ``block_manager`` free list, reference counts, fork and copy-on-write.
+* ``block_manager`` free list, reference counts, fork, copy-on-write and
+                    prefix caching across requests.
 * ``utilisation``   KV memory accounting: paged blocks versus contiguous
                     max-length reservation.
 

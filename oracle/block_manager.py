@@ -29,6 +29,26 @@ native manager, so the two are compared bit for bit):
   length and adds one reference to every block;
 * ``free(seq)`` drops one reference from each block of the sequence;
 * a failing call raises and leaves the state unchanged.
+
+Prefix caching across requests ([P3] second paragraph: blocks may be shared
+across the requests of a batch, not only within one; [P2] introduction and
+"From Contiguous Reserves to Paged KV Blocks": block tables make KV memory
+reusable and shareable).  The pages give no mechanism; the plainest reading,
+taken here: a block that a prompt fills completely is identified by its
+content, i.e. the whole token prefix up to the end of that block (the K/V of
+a position depend on every token before it).
+
+* ``allocate_prefix(seq, tokens)`` looks the prompt's full blocks up in
+  order, prefix by prefix, and stops at the first one not cached; each hit
+  joins the sequence's table with one more reference (a cached block whose
+  count had dropped to zero leaves the free list).  The other blocks are
+  taken from the front of the free list as in ``allocate``; every full one
+  is then entered in the cache under its prefix (replacing any older entry
+  for the same prefix).  Slots of tokens in hit blocks come back as -1: their
+  K/V are already in the pool, and the cache write skips them.
+* a freed block keeps its entry while it waits in the free list; it leaves
+  the cache when the free list hands it out again (to any allocation).
+* only prompt blocks are entered; blocks filled later by appends are not.
 """
 from __future__ import annotations
 
@@ -60,12 +80,20 @@ class BlockManager:
         self.ref = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        self.cache: dict[tuple, int] = {}      # token prefix of a full block -> block
+        self.key_of: dict[int, tuple] = {}     # block -> its prefix while cached
 
     # -- helpers ------------------------------------------------------------
     def _take(self) -> int:
         b = self.free.popleft()
         self.ref[b] = 1
+        self._uncache(b)
         return b
+
+    def _uncache(self, b: int) -> None:
+        key = self.key_of.pop(b, None)
+        if key is not None:
+            del self.cache[key]
 
     def _slot(self, seq: int, t: int) -> int:
         B = self.block_size
@@ -83,6 +111,46 @@ class BlockManager:
         self.tables[seq] = [self._take() for _ in range(need)]
         self.lens[seq] = num_tokens
         return [self._slot(seq, t) for t in range(num_tokens)]
+
+    def allocate_prefix(self, seq: int, tokens) -> tuple[list[int], int]:
+        """Allocate a prompt reusing cached full blocks; returns (slots with
+        -1 for cached tokens, number of cached tokens)."""
+        if seq in self.tables:
+            raise SeqExists(seq)
+        tokens = [int(x) for x in tokens]
+        B = self.block_size
+        n = len(tokens)
+        need = -(-n // B)
+        full = n // B
+        hits = []
+        for j in range(full):
+            b = self.cache.get(tuple(tokens[:(j + 1) * B]))
+            if b is None:
+                break
+            hits.append(b)
+        revived = sum(1 for b in hits if self.ref[b] == 0)
+        if need - len(hits) > len(self.free) - revived:
+            raise NoBlocks(need - len(hits))
+        for b in hits:
+            if self.ref[b] == 0:
+                self.free.remove(b)
+            self.ref[b] += 1
+        table = hits + [self._take() for _ in range(need - len(hits))]
+        for j in range(len(hits), full):
+            key = tuple(tokens[:(j + 1) * B])
+            old = self.cache.get(key)
+            if old is not None:
+                del self.key_of[old]
+            self.cache[key] = table[j]
+            self.key_of[table[j]] = key
+        self.tables[seq] = table
+        self.lens[seq] = n
+        cached = len(hits) * B
+        return [-1 if t < cached else self._slot(seq, t) for t in range(n)], cached
+
+    def num_cached(self) -> int:
+        """Blocks currently entered in the prefix cache (held or free)."""
+        return len(self.cache)
 
     def fork(self, parent: int, child: int) -> None:
         if parent not in self.tables:

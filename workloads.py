@@ -20,6 +20,9 @@ Workloads (sizes follow the decode shapes the library is built for):
              heads, head_dim 128, bf16, block 16 or 32, K given a large offset
              along the group's mean query at 8 positions per sequence so the
              softmax is peaked.
+* ``prefix`` chat-like requests sharing a few system prompts (or an earlier
+             request plus a new turn), at most 12 alive at once, with K/V
+             rows that depend only on the token prefix (prefix caching).
 
 Draw order for every batch: context lengths, then the physical block
 permutation (numpy PCG64 seeded with ``seed``); then q, K pool, V pool, new K,
@@ -328,3 +331,77 @@ def empty_pool(shape: Shape, num_blocks: int, seed: int, device="cpu"):
     k = torch.randn(*dims, generator=g, device=device, dtype=torch.float32).to(dt)
     v = torch.randn(*dims, generator=g, device=device, dtype=torch.float32).to(dt)
     return k, v
+
+
+# --------------------------------------------------------------------------
+# requests sharing prompt prefixes (for prefix caching across requests)
+# --------------------------------------------------------------------------
+@dataclass
+class PrefixWorkload:
+    shape: Shape
+    requests: list                    # token ids (np.int32 arrays), in arrival order
+    events: list                      # ("alloc", i) / ("free", i), in order
+    num_blocks: int
+    free_order: np.ndarray            # int32 [num_blocks]
+    seed: int
+
+
+def prefix_workload(shape: Shape | None = None, num_requests: int = 48, num_system: int = 4,
+                    system_range=(20, 300), suffix_range=(1, 120), vocab: int = 32000,
+                    live: int = 12, repeat_fraction: float = 0.25, seed: int = 7,
+                    num_blocks: int | None = None) -> PrefixWorkload:
+    """Chat-like requests: each is one of a few system prompts (drawn with
+    skewed weights) followed by its own suffix, or, with probability
+    ``repeat_fraction``, an earlier request followed by a new turn.  At most
+    ``live`` requests are held at once: before a request arrives a random live
+    one finishes when the limit is reached.  The default pool holds about
+    1.5 times the live requests' blocks, so freed blocks are reused and
+    retained prefixes are eventually handed out again."""
+    sh = shape if shape is not None else SHAPES["gqa8b"]
+    rng = np.random.default_rng(seed)
+    systems = [rng.integers(0, vocab, size=int(rng.integers(system_range[0], system_range[1],
+                                                            endpoint=True))).astype(np.int32)
+               for _ in range(num_system)]
+    weights = rng.dirichlet(np.full(num_system, 0.7))
+    requests, events, alive = [], [], []
+    for i in range(num_requests):
+        suffix = rng.integers(0, vocab, size=int(rng.integers(suffix_range[0], suffix_range[1],
+                                                              endpoint=True))).astype(np.int32)
+        if requests and rng.random() < repeat_fraction:
+            base = requests[int(rng.integers(0, len(requests)))]
+        else:
+            base = systems[int(rng.choice(num_system, p=weights))]
+        requests.append(np.concatenate([base, suffix]).astype(np.int32))
+        if len(alive) >= live:
+            j = alive.pop(int(rng.integers(0, len(alive))))
+            events.append(("free", j))
+        events.append(("alloc", i))
+        alive.append(i)
+    B = sh.block_size
+    if num_blocks is None:
+        biggest = sorted((_ceil_div(len(r), B) for r in requests), reverse=True)[:live]
+        num_blocks = int(math.ceil(1.5 * sum(biggest))) + live * 4
+    perm = rng.permutation(num_blocks).astype(np.int32)
+    return PrefixWorkload(shape=sh, requests=requests, events=events, num_blocks=num_blocks,
+                          free_order=perm, seed=seed)
+
+
+def prefix_kv_rows(tokens, shape: Shape, seed: int, device="cpu"):
+    """Synthetic K and V rows [n, Hkv, D] for a prompt, row t a function of
+    (seed, tokens[0..t]) only -- as a model's K/V at a position depend on the
+    whole prefix -- so requests with equal prefixes get bit-equal rows.  Row t
+    is N(0, 1) drawn by a PCG64 generator seeded with (seed, running CRC-32 of
+    the prefix), rounded to nearest-even into the storage dtype."""
+    import zlib
+    dims = (shape.num_kv_heads, shape.head_dim)
+    n = len(tokens)
+    k = np.empty((n,) + dims, dtype=np.float32)
+    v = np.empty((n,) + dims, dtype=np.float32)
+    crc = 0
+    for t, tok in enumerate(np.asarray(tokens, dtype=np.int32).tolist()):
+        crc = zlib.crc32(np.int32(tok).tobytes(), crc)
+        g = np.random.default_rng([int(seed), crc])
+        k[t] = g.standard_normal(dims, dtype=np.float32)
+        v[t] = g.standard_normal(dims, dtype=np.float32)
+    dt = TORCH_DTYPES[shape.dtype]
+    return torch.from_numpy(k).to(dt).to(device), torch.from_numpy(v).to(dt).to(device)
