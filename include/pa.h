@@ -241,8 +241,9 @@ int pa_device_error(unsigned *flags, int clear);
  *
  * Policy: the free list is first-in-first-out, initialised from free_order
  * (NULL = 0 .. num_blocks-1); blocks whose reference count drops to zero go
- * to its back.  Every failing call returns a negative pa_status and leaves
- * the manager unchanged.
+ * to its back (a prefix-cache hit may take a block out of its middle).
+ * Every failing call returns a negative pa_status and leaves the manager
+ * unchanged.
  * ---------------------------------------------------------------------- */
 typedef struct pa_bm pa_bm;
 
@@ -276,8 +277,42 @@ int pa_bm_append_slot(pa_bm *bm, int64_t seq, int64_t *slot_out, int32_t *cow_sr
 int pa_bm_append_slots(pa_bm *bm, const int64_t *seqs, int n, int64_t *slots_out,
                        int64_t *cow_pairs_out, int *num_cow_out);
 
-/* Drop the sequence: one reference less on each of its blocks. */
+/* Drop the sequence: one reference less on each of its blocks.  A block
+ * that reaches zero goes to the back of the free list; if it holds a cached
+ * prompt prefix (pa_bm_allocate_prefix) it stays in the cache until the free
+ * list hands it out again. */
 int pa_bm_free(pa_bm *bm, int64_t seq);
+
+/*
+ * Prefix caching across requests ([P3] second paragraph: blocks may be
+ * shared across the requests of a batch; [P2] introduction and "From
+ * Contiguous Reserves to Paged KV Blocks": block tables make KV memory
+ * reusable and shareable).  The pages give no mechanism; the one here:
+ *
+ * A block that a prompt fills completely is identified by its whole token
+ * prefix tokens[0 .. (j+1)*block_size) (compared exactly, never by hash
+ * alone).  New sequence `seq` with the prompt tokens[0 .. num_tokens)
+ * (int32 token ids, host memory): its full blocks are looked up in order and
+ * the lookup stops at the first prefix not cached; each hit joins the table
+ * with one more reference (a cached block waiting in the free list leaves
+ * it).  The remaining ceil(num_tokens / block_size) - hits blocks come from
+ * the front of the free list as in pa_bm_allocate, and each of them that is
+ * full is entered in the cache under its prefix (replacing an older entry
+ * for the same prefix).  slots_out (int64 [num_tokens], may be NULL) gets -1
+ * for the tokens of hit blocks -- their K/V are already in the pool and
+ * pa_reshape_and_cache skips negative slots -- and the slot of every other
+ * token; *num_cached_out (may be NULL) = hits * block_size.  Only prompt
+ * blocks are entered; blocks filled later by appends are not.  Cached
+ * blocks are full, so appends never write or copy them.
+ *
+ * A block leaves the cache when any call takes it from the free list for
+ * new content.  PA_ERR_SEQ if seq exists; PA_ERR_NO_BLOCKS (nothing
+ * changed) if the free list, less the hits it holds, is too short.
+ */
+int pa_bm_allocate_prefix(pa_bm *bm, int64_t seq, const int32_t *tokens, int num_tokens,
+                          int64_t *slots_out, int *num_cached_out);
+/* Number of blocks entered in the prefix cache (held or free). */
+int pa_bm_num_cached(const pa_bm *bm);
 
 /* Copy the sequence's block table into out[0 .. cap) (*n_out = its length);
  * PA_ERR_ARG if cap is too small. */

@@ -95,6 +95,8 @@ def _declare(L):
         "pa_bm_ref_count": (i32, [vp, c.c_int32]),
         "pa_bm_num_seqs": (i32, [vp]),
         "pa_bm_stats": (i32, [vp, c.POINTER(BmStats)]),
+        "pa_bm_allocate_prefix": (i32, [vp, i64, P32, i32, P64, c.POINTER(c.c_int)]),
+        "pa_bm_num_cached": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -348,6 +350,23 @@ class BlockManager:
         slots = np.empty(max(num_tokens, 0), dtype=np.int64)
         _check(lib().pa_bm_allocate(self._h, seq, num_tokens, _p64(slots)), "pa_bm_allocate")
         return slots
+
+    def allocate_prefix(self, seq: int, tokens, slots_out=None):
+        """Allocate a prompt of token ids, reusing cached full blocks whose
+        whole token prefix matches.  Returns (slots int64 [n], -1 for the
+        cached tokens; number of cached tokens)."""
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = toks.shape[0]
+        slots = (np.empty(n, dtype=np.int64) if slots_out is None
+                 else _out(slots_out, (n,), np.int64))
+        got = ctypes.c_int(0)
+        _check(lib().pa_bm_allocate_prefix(self._h, seq, _p32(toks), n, _p64(slots),
+                                           ctypes.byref(got)), "pa_bm_allocate_prefix")
+        return slots, int(got.value)
+
+    def num_cached(self) -> int:
+        """Blocks entered in the prefix cache (held by a sequence or free)."""
+        return lib().pa_bm_num_cached(self._h)
 
     def fork(self, parent: int, child: int) -> None:
         _check(lib().pa_bm_fork(self._h, parent, child), "pa_bm_fork")
