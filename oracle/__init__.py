@@ -11,7 +11,8 @@ Everything is written to be checked by eye against the pages it follows:
 * ``fp``            exact decoding of fp16 / bf16 storage bits to float64.
 * ``attention``     gather a sequence's logical K/V through its block table,
                     then softmax(q K^T * scale) V in float64; the split-context
-                    partial/merge algebra.
+                    partial/merge algebra; the causal multi-token form
+                    of a chunked prefill.
 * ``cache_ops``     reshape_and_cache (scatter of new K/V into their slots) and
                     copy_blocks (copy-on-write block copies), on raw bits.
 * ``block_manager`` free list, reference counts, fork, copy-on-write and

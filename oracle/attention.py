@@ -105,3 +105,43 @@ def split_context_attention(qvec, K, V, scale: float, partition: int) -> np.ndar
     parts = [partial_attention(qvec, K[a:a + partition], V[a:a + partition], scale)
              for a in range(0, L, partition)]
     return merge_partials(parts)
+
+
+# ----------------------------------------------------------------------------
+# chunked prefill: several new tokens of a sequence at once
+# ----------------------------------------------------------------------------
+
+def paged_prefill_attention(q_bits, k_cache_bits, v_cache_bits, block_tables, context_lens,
+                            query_start, scale: float, num_kv_heads: int, block_size: int,
+                            dtype: str, seqs=None) -> np.ndarray:
+    """Attention of a chunk of new tokens per sequence over the paged cache.
+
+    Not on the pages beyond their statement that attention runs block by
+    block over non-contiguous blocks ([P3] second paragraph) and that the
+    KV cache is filled as tokens arrive ([P1] section 2); written here as the
+    plainest multi-token form of steps 1-4.  Sequence s owns the query rows
+    query_start[s] .. query_start[s+1]-1 of ``q_bits`` [T, Hq, D]: its last
+    C_s = query_start[s+1] - query_start[s] tokens, whose K/V are already in
+    the cache (the cache write comes first, as in decode), so its context
+    holds L_s = context_lens[s] >= C_s tokens.  Row i (0 <= i < C_s) is the
+    token at position p = L_s - C_s + i and, causally, attends to positions
+    0 .. p only.  C_s = 1 is a decode step.  Returns out [T, Hq, D] float64
+    (rows of sequences not in ``seqs`` left NaN)."""
+    T, Hq, D = q_bits.shape
+    assert Hq % num_kv_heads == 0
+    G = Hq // num_kv_heads
+    out = np.full((T, Hq, D), np.nan, dtype=np.float64)
+    todo = range(len(context_lens)) if seqs is None else seqs
+    for s in todo:
+        a, b = int(query_start[s]), int(query_start[s + 1])
+        C, L = b - a, int(context_lens[s])
+        assert 0 <= C <= L
+        for kh in range(num_kv_heads):
+            K = gather_logical_kv(k_cache_bits, block_tables[s], L, kh, block_size, dtype)
+            V = gather_logical_kv(v_cache_bits, block_tables[s], L, kh, block_size, dtype)
+            for i in range(C):
+                p = L - C + i
+                qs = decode(q_bits[a + i], dtype)
+                for h in range(kh * G, (kh + 1) * G):
+                    out[a + i, h] = softmax_attention(qs[h], K[:p + 1], V[:p + 1], scale)
+    return out

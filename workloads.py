@@ -405,3 +405,99 @@ def prefix_kv_rows(tokens, shape: Shape, seed: int, device="cpu"):
         v[t] = g.standard_normal(dims, dtype=np.float32)
     dt = TORCH_DTYPES[shape.dtype]
     return torch.from_numpy(k).to(dt).to(device), torch.from_numpy(v).to(dt).to(device)
+
+
+# --------------------------------------------------------------------------
+# chunked prefill: several new tokens per sequence
+# --------------------------------------------------------------------------
+@dataclass
+class PrefillBatch:
+    shape: Shape
+    context_lens: np.ndarray          # int32 [S], tokens after this chunk
+    chunk_lens: np.ndarray            # int32 [S], new tokens this step (<= context_lens)
+    query_start: np.ndarray           # int32 [S+1], running sum of chunk_lens
+    block_tables: np.ndarray          # int32 [S, max_blocks_per_seq], -1 = unused
+    free_order: np.ndarray            # int32 [num_blocks]
+    num_blocks: int
+    q: torch.Tensor                   # [T, Hq, D], T = sum(chunk_lens)
+    k_cache: torch.Tensor             # [num_blocks, Hkv, B, D]
+    v_cache: torch.Tensor
+    k_new: torch.Tensor               # [T, Hkv, D] the chunk's tokens
+    v_new: torch.Tensor
+    scale: float
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+
+def make_prefill_batch(shape: Shape, context_lens, chunk_lens, seed: int, *, device="cpu",
+                       spare_fraction: float = 0.10, max_blocks_per_seq: int | None = None,
+                       poison: str | None = None) -> PrefillBatch:
+    """Draw one chunked-prefill batch.  Sequence s already holds
+    context_lens[s] - chunk_lens[s] tokens and adds chunk_lens[s] this step.
+    Blocks are consecutive runs of one permutation, sequence by sequence, as
+    a first-in-first-out manager seeded with ``free_order`` hands them out
+    when each sequence is allocated and then extended by its chunk before the
+    next one.  Draw order: permutation (numpy), then q, K pool, V pool, new K,
+    new V (torch generator), N(0, 1) rounded into the storage dtype;
+    ``poison='nan'`` as for decode batches."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(context_lens, dtype=np.int32)
+    chunks = np.asarray(chunk_lens, dtype=np.int32)
+    assert lens.shape == chunks.shape and (chunks >= 0).all() and (chunks <= lens).all()
+    B = shape.block_size
+    nb = [_ceil_div(int(x), B) for x in lens]
+    used = int(sum(nb))
+    num_blocks = max(1, int(math.ceil(used * (1.0 + spare_fraction))))
+    maxb = max_blocks_per_seq if max_blocks_per_seq is not None else max(1, max(nb, default=1))
+    perm = rng.permutation(num_blocks).astype(np.int32)
+    tables = np.full((len(lens), maxb), -1, dtype=np.int32)
+    off = 0
+    for s, n in enumerate(nb):
+        tables[s, :n] = perm[off:off + n]
+        off += n
+    qstart = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    T = int(qstart[-1])
+    dt = TORCH_DTYPES[shape.dtype]
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    Hq, Hkv, D = shape.num_q_heads, shape.num_kv_heads, shape.head_dim
+
+    def draw(*dims):
+        return torch.randn(*dims, generator=g, device=device, dtype=torch.float32).to(dt)
+
+    q = draw(T, Hq, D)
+    k_cache = draw(num_blocks, Hkv, B, D)
+    v_cache = draw(num_blocks, Hkv, B, D)
+    k_new = draw(T, Hkv, D)
+    v_new = draw(T, Hkv, D)
+    if poison == "nan":
+        valid = torch.zeros(num_blocks, B, dtype=torch.bool)
+        for s, n in enumerate(nb):
+            for j in range(n):
+                valid[int(tables[s, j]), :min(B, int(lens[s]) - j * B)] = True
+        mask = (~valid).to(device)[:, None, :, None].expand(num_blocks, Hkv, B, D)
+        nan = torch.tensor(NAN_BITS[shape.dtype], dtype=torch.int16, device=device).view(dt)
+        k_cache[mask] = nan
+        v_cache[mask] = nan
+    elif poison is not None:
+        raise ValueError(poison)
+    return PrefillBatch(shape=shape, context_lens=lens, chunk_lens=chunks, query_start=qstart,
+                        block_tables=tables, free_order=perm, num_blocks=num_blocks, q=q,
+                        k_cache=k_cache, v_cache=v_cache, k_new=k_new, v_new=v_new,
+                        scale=1.0 / math.sqrt(D))
+
+
+def prefill_lens(rng: np.random.Generator, num_seqs: int = 16, chunk: int = 512,
+                 max_len: int = 4096):
+    """Chunked-prefill mix: every sequence adds a chunk of ``chunk`` tokens on
+    top of 0 .. max_len - chunk tokens already cached (uniform, in whole
+    chunks, as a long prompt processed chunk by chunk)."""
+    before = chunk * rng.integers(0, max_len // chunk, size=num_seqs)
+    chunks = np.full(num_seqs, chunk, dtype=np.int32)
+    return (before + chunks).astype(np.int32), chunks
