@@ -224,6 +224,48 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
                    pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * Chunked-prefill attention: several new tokens per sequence attend over the
+ * paged cache at once ("Can OS paging techniques reduce LLM serving memory
+ * waste?", second paragraph: attention block by block over non-contiguous
+ * blocks; "Why OS Virtual Memory Paging Saved LLM Inference: The vLLM
+ * Breakthrough", section 2: the cache fills as tokens arrive).  The pages
+ * describe only the single-token case; this is its causal multi-token form.
+ *
+ * Sequence s owns query rows query_start[s] .. query_start[s+1]-1 of q: its
+ * last C_s = query_start[s+1] - query_start[s] tokens, already written to the
+ * cache (pa_reshape_and_cache first, as for decode), so context_lens[s] =
+ * L_s >= C_s.  Row i is the token at position L_s - C_s + i and attends to
+ * positions 0 .. L_s - C_s + i:
+ *   out[t, h, :] = softmax(scale * q[t, h, :] . K_s[0..p]) V_s[0..p]
+ * with kv head h / (num_q_heads / num_kv_heads).
+ *
+ *   out          fp32 [num_tokens, num_q_heads, head_dim] (device, 16-byte aligned)
+ *   q            cache dtype [num_tokens, num_q_heads, head_dim] (device, 16-byte aligned)
+ *   k/v_cache    [num_blocks, num_kv_heads, block_size, head_dim] (device)
+ *   block_tables int32 [num_seqs, max_blocks_per_seq] (device)
+ *   context_lens int32 [num_seqs] (device), tokens including the chunk
+ *   query_start  int32 [num_seqs + 1] (device), non-decreasing, query_start[0] = 0,
+ *                query_start[num_seqs] = num_tokens
+ *   max_query_len host upper bound of every C_s (sizes the grid; longer chunks
+ *                are not computed)
+ * head_dim 64 or 128, block_size 16 or 32, group size up to 16, fp16 or
+ * bf16.  Runs on the tensor cores (tcgen05): P is rounded to the cache dtype
+ * before P.V, so the result carries that rounding (relative 2^-9 per weight
+ * for bf16, 2^-12 for fp16) besides the fp32 accumulation.  No workspace,
+ * nothing allocated.  A chunk longer than its context, a context longer
+ * than the table, or rows outside [0, num_tokens) set PA_DEVERR_CONTEXT_LEN
+ * and leave that sequence's rows unwritten; block ids outside the pool are skipped and set
+ * PA_DEVERR_BLOCK_ID.  Rows of a sequence whose C_s is 0 are none.
+ */
+int pa_paged_prefill_attention(float *out, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, const int32_t *query_start,
+                               float scale, int num_kv_heads, int num_seqs, int num_tokens,
+                               int num_q_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int max_query_len, int num_blocks,
+                               pa_dtype dtype, pa_stream_t stream);
+
+/*
  * Read the sticky device error word of the current device into *flags
  * (PA_DEVERR_* bits; may be NULL), clearing it if `clear` is non-zero.
  * Synchronises the device.  Returns PA_OK when no bit is set,

@@ -79,6 +79,8 @@ def _declare(L):
         "pa_decode_step": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                  i32, i32, i32, i32, vp, sz, vp]),
         "pa_decode_tuning": (i32, [i32, i32, i32]),
+        "pa_paged_prefill_attention": (i32, [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32,
+                                             i32, i32, i32, i32, i32, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
         "pa_device_error": (i32, [c.POINTER(c.c_uint), i32]),
         "pa_bm_create": (vp, [i32, i32, P32]),
@@ -267,6 +269,33 @@ def pa_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, context
         int(max_context_len), NB, _dtype_code(k_cache), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_decode_step")
+    return out
+
+
+def pa_paged_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens,
+                               query_start, scale, num_kv_heads, max_query_len, stream=None):
+    """Chunked prefill: query row t of sequence s (rows query_start[s] ..
+    query_start[s+1]-1, the sequence's last tokens, already in the cache) at
+    position p attends to positions 0..p of its sequence.  q [T, Hq, D],
+    out [T, Hq, D] fp32; max_query_len bounds every chunk (host int)."""
+    torch = _torch()
+    T, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    if Hkv != num_kv_heads or D2 != D:
+        raise ValueError("q / cache shapes disagree")
+    if tuple(out.shape) != (T, Hq, D):
+        raise ValueError("out must be [num_tokens, num_q_heads, head_dim]")
+    S = int(context_lens.shape[0])
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or query_start.shape != (S + 1,):
+        raise ValueError("block_tables [S, max_blocks] / query_start [S + 1] expected")
+    st = lib().pa_paged_prefill_attention(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), float(scale), Hkv, S, T, Hq, D, B,
+        int(block_tables.shape[1]), int(max_query_len), NB, _dtype_code(k_cache),
+        _stream(stream))
+    _check(st, "pa_paged_prefill_attention")
     return out
 
 

@@ -19,7 +19,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 
 CU_SOURCES = ["pa_kernels.cu"]
 CPP_SOURCES = ["block_manager.cpp"]
-HEADERS = ["pa_device.cuh", "decode_attention.cuh", "cache_ops.cuh"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

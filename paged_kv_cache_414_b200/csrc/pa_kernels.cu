@@ -14,6 +14,7 @@
 #include "pa_device.cuh"
 #include "cache_ops.cuh"
 #include "decode_attention.cuh"
+#include "prefill_attention.cuh"
 
 namespace {
 
@@ -262,6 +263,93 @@ int dispatch_shape(const DecodeArgs &a, int dev, int sms) {
   return dispatch_group<T, 64, 32>(a, dev, sms);
 }
 
+// ---------------------------------------------------------------- chunked prefill
+
+// Q [T, Hq, D] as a 3-D map (D, Hq, T); a box is 64 columns x the G heads of
+// one kv head x TQ tokens, i.e. 128 query rows ordered (token, head).
+bool encode_query_map(CUtensorMap *m, const void *q, int T, int Hq, int D, int G, int tq) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)tq};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(q), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct PrefillArgs {
+  float *out;
+  const void *q, *k_cache, *v_cache;
+  const int32_t *block_tables, *context_lens, *query_start;
+  float scale;
+  int num_kv_heads, num_seqs, num_tokens, num_q_heads, head_dim, block_size, max_blocks,
+      max_query_len, num_blocks;
+  cudaStream_t stream;
+};
+
+template <typename T, int D, int B>
+int launch_prefill(const PrefillArgs &a, int dev) {
+  using L = pa::PrefillSmem<D>;
+  auto kern = pa::paged_prefill_kernel<T, D, B>;
+  static std::atomic<int> attr_set[kMaxDevices];
+  if (!attr_set[dev].load()) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    attr_set[dev].store(1);
+  }
+  const int G = a.num_q_heads / a.num_kv_heads;
+  const int tq = pa::kPfRows / G;
+  CUtensorMap qmap, kmap, vmap;
+  const long long rows = (long long)a.num_blocks * a.num_kv_heads * B;
+  if (!encode_query_map(&qmap, a.q, a.num_tokens, a.num_q_heads, D, G, tq) ||
+      !encode_pool_map(&kmap, a.k_cache, rows, D, B) ||
+      !encode_pool_map(&vmap, a.v_cache, rows, D, B))
+    return PA_ERR_CUDA;
+  pa::PrefillParams p;
+  p.out = a.out;
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  p.query_start = a.query_start;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.num_seqs = a.num_seqs;
+  p.num_tokens = a.num_tokens;
+  p.num_q_heads = a.num_q_heads;
+  p.num_kv_heads = a.num_kv_heads;
+  p.group = G;
+  p.max_blocks = a.max_blocks;
+  p.num_blocks = a.num_blocks;
+  p.tq = tq;
+  p.q_tiles = (a.max_query_len + tq - 1) / tq;
+  const long long nx = (long long)p.q_tiles * a.num_seqs;
+  if (nx >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nx, (unsigned)a.num_kv_heads);
+  cfg.blockDim = dim3(pa::kPfThreads);
+  cfg.dynamicSmemBytes = L::BYTES;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, qmap, kmap, vmap, p) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+template <typename T>
+int dispatch_prefill(const PrefillArgs &a, int dev) {
+  if (a.head_dim == 128 && a.block_size == 16) return launch_prefill<T, 128, 16>(a, dev);
+  if (a.head_dim == 128 && a.block_size == 32) return launch_prefill<T, 128, 32>(a, dev);
+  if (a.head_dim == 64 && a.block_size == 16) return launch_prefill<T, 64, 16>(a, dev);
+  return launch_prefill<T, 64, 32>(a, dev);
+}
+
 bool supported_shape(int head_dim, int block_size) {
   return (head_dim == 64 || head_dim == 128) && (block_size == 16 || block_size == 32);
 }
@@ -498,6 +586,38 @@ int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_
                num_blocks,   scratch,     kNoAllocScratchBytes, (cudaStream_t)stream};
   if (dtype == PA_BF16) return dispatch_shape<__nv_bfloat16>(a, dev, sms);
   return dispatch_shape<__half>(a, dev, sms);
+}
+
+int pa_paged_prefill_attention(float *out, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, const int32_t *query_start,
+                               float scale, int num_kv_heads, int num_seqs, int num_tokens,
+                               int num_q_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int max_query_len, int num_blocks,
+                               pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_kv_heads <= 0 ||
+      num_q_heads <= 0 || head_dim <= 0 || block_size <= 0)
+    return PA_ERR_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_ARG;
+  if (!supported_shape(head_dim, block_size) || num_q_heads / num_kv_heads > 16)
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (max_blocks_per_seq <= 0 || num_blocks <= 0) return PA_ERR_ARG;
+  if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
+    return PA_ERR_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4))
+    return PA_ERR_ARG;
+  int dev;
+  if (current_device(&dev) != PA_OK || dev >= kMaxDevices) return PA_ERR_CUDA;
+  PrefillArgs a{out,          q,           k_cache,       v_cache,     block_tables,
+                context_lens, query_start, scale,         num_kv_heads, num_seqs,
+                num_tokens,   num_q_heads, head_dim,      block_size,  max_blocks_per_seq,
+                max_query_len, num_blocks, (cudaStream_t)stream};
+  if (dtype == PA_BF16) return dispatch_prefill<__nv_bfloat16>(a, dev);
+  return dispatch_prefill<__half>(a, dev);
 }
 
 int pa_decode_tuning(int nstage, int ctas_per_sm, int min_tiles_per_warp) {

@@ -1,0 +1,422 @@
+// Chunked-prefill attention over the paged KV cache, on the fifth-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// What it computes ("Can OS paging techniques reduce LLM serving memory
+// waste?", second paragraph: attention runs block by block over blocks that
+// need not be contiguous; "Why OS Virtual Memory Paging Saved LLM Inference:
+// The vLLM Breakthrough", section 2: the KV cache fills as tokens arrive, the
+// block table maps logical to physical blocks).  Sequence s adds a chunk of
+// C_s tokens whose K/V are already in the cache; its context holds
+// L_s >= C_s tokens.  Chunk token i sits at position L_s - C_s + i and attends
+// causally to positions 0 .. L_s - C_s + i:
+//   out[t, h] = softmax(scale * q[t, h] . K_s[0..p]) V_s[0..p].
+//
+// Work split: one CTA per (sequence, kv head, query tile).  A query tile is
+// 128 rows = TQ = 128 / G chunk tokens x the G query heads that share the kv
+// head, so every K/V tile fetched from the pool serves all 128 rows.  Keys go
+// in tiles of 128 positions (8 blocks of 16 or 4 of 32), fetched by TMA
+// straight from their physical blocks into 128-byte-swizzled shared memory.
+//
+//   warp 0      TMA producer: Q once, then K/V tiles into a two-stage ring.
+//   warp 1      owns the tensor memory; one lane issues the MMAs:
+//                 S_j = Q K_j^T    (M 128, N 128 keys, K = head_dim), into one
+//                                  of two S buffers, so S_{j+1} runs while the
+//                                  softmax works on S_j;
+//                 O  += P_j V_j    (M 128, N = head_dim, K 128 keys).
+//   warps 2-5   softmax, one thread per row (tensor-memory lane): online
+//               maximum and sum in fp32; P_j goes to tensor memory, where the
+//               P.V MMA reads it as its A operand.  For bf16, P = P_hi + P_lo
+//               (both bf16, two MMAs), so P carries about 2^-17 relative
+//               rounding instead of bf16's 2^-9; for fp16 one fp16 P whose
+//               rounded weights are also what the sum adds.  O is rescaled in
+//               tensor memory when the row maximum moves; the epilogue writes
+//               out = O / l.
+//
+// Tensor memory (512 columns): S buffers at 0 and 128, O at 256 (head_dim
+// columns), P_hi at 384 and P_lo at 448 (64 columns each: 128 16-bit
+// weights per row, two per column).
+//
+// Every wait is bounded: on time-out a shared abort flag stops every role,
+// PA_DEVERR_TIMEOUT is set, copies and MMAs in flight are waited for (again
+// bounded) and the tensor memory is freed.
+#pragma once
+
+#include <math.h>
+
+#include "umma.cuh"
+
+namespace pa {
+
+struct PrefillParams {
+  float *out;                    // [T, Hq, D]
+  const int32_t *block_tables;   // [S, max_blocks]
+  const int32_t *context_lens;   // [S]
+  const int32_t *query_start;    // [S + 1]
+  float scale_log2;              // scale * log2(e)
+  int num_seqs, num_tokens, num_q_heads, num_kv_heads, group, max_blocks, num_blocks;
+  int q_tiles;                   // query tiles per sequence in the grid
+  int tq;                        // chunk tokens per query tile (128 / group)
+};
+
+constexpr int kPfRows = 128;      // query rows per CTA
+constexpr int kPfKeys = 128;      // keys per K/V tile
+constexpr int kPfThreads = 192;   // producer warp, MMA warp, 4 softmax warps
+constexpr uint32_t kPfTmemCols = 512;
+constexpr uint64_t kPfWaitLimitNs = 2000000000ull;
+
+template <int D>
+struct PrefillSmem {
+  static constexpr int NCH = D / 64;                  // 64-column chunks of a row
+  static constexpr int REGION = kPfRows * 128;        // one 64-column chunk of 128 rows
+  static constexpr int Q_BYTES = NCH * REGION;
+  static constexpr int KV_BYTES = NCH * kPfKeys * 128;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;       // two stages
+  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // two stages
+  static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
+  static constexpr int BYTES = OFF_BAR + 128 + 1024;  // barriers + alignment slack
+};
+
+// Bounded wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kPfWaitLimitNs) {
+      *abort = 1;
+      flag_error(PA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Rounding of the softmax weights to the MMA's input type.
+template <typename T>
+struct PfPack;
+template <>
+struct PfPack<__nv_bfloat16> {
+  static constexpr bool kBf16 = true;
+  static constexpr bool kSplit = true;     // P = hi + lo
+  // (a, b) -> packed hi pair, packed lo pair (the rounding remainders)
+  __device__ __forceinline__ static void split2(float a, float b, uint32_t *hi, uint32_t *lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    float2 f = __bfloat1622float2(h);
+    __nv_bfloat162 r = __floats2bfloat162_rn(a - f.x, b - f.y);
+    *hi = *reinterpret_cast<uint32_t *>(&h);
+    *lo = *reinterpret_cast<uint32_t *>(&r);
+  }
+  __device__ __forceinline__ static uint32_t round2(float a, float b, float *sum) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    float2 f = __bfloat1622float2(h);
+    *sum += f.x + f.y;
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
+};
+template <>
+struct PfPack<__half> {
+  static constexpr bool kBf16 = false;
+  static constexpr bool kSplit = false;    // one fp16 P
+  __device__ __forceinline__ static void split2(float, float, uint32_t *, uint32_t *) {}
+  // round two weights to fp16; return the packed pair and add the rounded
+  // values to *sum (so the normalisation matches what the MMA multiplies)
+  __device__ __forceinline__ static uint32_t round2(float a, float b, float *sum) {
+    __half2 h = __floats2half2_rn(a, b);
+    float2 f = __half22float2(h);
+    *sum += f.x + f.y;
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
+};
+
+template <typename T, int D, int B>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap,
+                         const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
+  using L = PrefillSmem<D>;
+  constexpr int NCH = L::NCH;
+  constexpr int BPT = kPfKeys / B;                    // blocks per K/V tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem + L::OFF_Q;
+  uint8_t *sK = smem + L::OFF_K;
+  uint8_t *sV = smem + L::OFF_V;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
+  uint64_t *full = bars + 0;       // [2] K/V stage landed
+  uint64_t *empty = bars + 2;      // [2] K/V stage consumed
+  uint64_t *q_full = bars + 4;     // Q landed
+  uint64_t *s_full = bars + 5;     // [2] S buffer written
+  uint64_t *p_full = bars + 7;     // P written and O rescaled (128 arrivals)
+  uint64_t *o_done = bars + 8;     // O += P V done
+  uint64_t *drain = bars + 9;      // every MMA done (before freeing tensor memory)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+  volatile int *abort = reinterpret_cast<volatile int *>(bars + 11);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.x % p.num_seqs;
+  const int qt = p.q_tiles - 1 - blockIdx.x / p.num_seqs;   // longest tiles first
+  const int kh = blockIdx.y;
+  const int G = p.group;
+
+  grid_dependency_wait();     // the chunk's cache write may be the kernel before
+  const int q0 = __ldg(p.query_start + s);
+  const int C = __ldg(p.query_start + s + 1) - q0;
+  const int Lc = __ldg(p.context_lens + s);
+  const int tok0 = qt * p.tq;
+  if (C < 0 || C > Lc || Lc > p.max_blocks * B || q0 < 0 || q0 + C > p.num_tokens) {
+    if (threadIdx.x == 0 && kh == 0 && qt == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
+    return;
+  }
+  if (tok0 >= C) return;                               // uniform over the CTA
+  const int ntok = min(p.tq, C - tok0);
+  const int pos_max = Lc - C + tok0 + ntok - 1;        // last position any row sees
+  const int n_tiles = pos_max / kPfKeys + 1;
+  const int nb_used = pos_max / B + 1;                 // blocks holding positions 0..pos_max
+  const int rows_q = p.tq * G;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&s_full[i], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kPfTmemCols);
+    tmem_relinquish();
+  }
+  if (rows_q < kPfRows) {     // Q rows no chunk token fills: zeros, not stale bits
+    for (int i = threadIdx.x; i < NCH * (kPfRows - rows_q) * 8; i += kPfThreads) {
+      const int c = i / ((kPfRows - rows_q) * 8), rem = i % ((kPfRows - rows_q) * 8);
+      *reinterpret_cast<uint4 *>(sQ + c * L::REGION + (rows_q + rem / 8) * 128 + (rem % 8) * 16) =
+          make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 2 * kPfKeys, tP = tmem + 3 * kPfKeys,
+                 tPlo = tP + kPfKeys / 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+      mbar_arrive_expect_tx(q_full, NCH * 128 * rows_q);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_3d(sQ + c * L::REGION, &qmap, c * 64, kh * G, q0 + tok0, q_full);
+      const int32_t *table = p.block_tables + (size_t)s * p.max_blocks;
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !pf_wait(&empty[st], ((j >> 1) - 1) & 1, abort)) break;
+        const int b0 = j * BPT;
+        const int nb = min(BPT, nb_used - b0);
+        int ids[BPT];
+        int nvalid = 0;
+#pragma unroll
+        for (int b = 0; b < BPT; ++b) {
+          ids[b] = -1;
+          if (b < nb) {
+            const int id = __ldg(table + b0 + b);
+            if (id >= 0 && id < p.num_blocks) {
+              ids[b] = id;
+              ++nvalid;
+            } else {
+              flag_error(PA_DEVERR_BLOCK_ID);
+            }
+          }
+        }
+        mbar_arrive_expect_tx(&full[st], nvalid * 2 * NCH * B * 128);
+#pragma unroll
+        for (int b = 0; b < BPT; ++b) {
+          if (ids[b] < 0) continue;
+          const int row = (ids[b] * p.num_kv_heads + kh) * B;
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            const int off = st * L::KV_BYTES + c * kPfKeys * 128 + b * B * 128;
+            tma_load_2d(sK + off, &kmap, c * 64, row, &full[st]);
+            tma_load_2d(sV + off, &vmap, c * 64, row, &full[st]);
+          }
+        }
+        issued = j + 1;
+      }
+      // copies still in flight must land before the CTA exits
+      for (int j = max(0, issued - 2); j < issued; ++j)
+        mbar_wait_bounded(&full[j & 1], (j >> 1) & 1, kPfWaitLimitNs);
+      mbar_wait_bounded(q_full, 0, kPfWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr bool kBf = PfPack<T>::kBf16;
+      const uint32_t idS = umma_idesc_f16(kBf, kPfRows, kPfKeys, false, false);
+      const uint32_t idO = umma_idesc_f16(kBf, kPfRows, D, false, true);
+      const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+      auto issue_s = [&](int j) {
+        const uint32_t k0 = aK + (j & 1) * L::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kPfKeys * 128) + (kk & 3) * 32;
+          const uint64_t da = umma_desc_sw128(aQ + (kk >> 2) * L::REGION + (kk & 3) * 32, 16, 1024);
+          const uint64_t db = umma_desc_sw128(k0 + off, 16, 1024);
+          umma_f16_ss(tS + (j & 1) * kPfKeys, da, db, idS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[j & 1]);
+      };
+      bool ok = pf_wait(q_full, 0, abort) && pf_wait(&full[0], 0, abort);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles) {
+          if (!pf_wait(&full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort)) break;
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        if (!pf_wait(p_full, j & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t v0 = aV + (j & 1) * L::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
+          // 16 keys: 8 columns of P, 16 rows of V
+          const uint64_t db = umma_desc_sw128(v0 + kk * 16 * 128, kPfKeys * 128, 1024);
+          umma_f16_ts(tO, tP + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          if (PfPack<T>::kSplit) umma_f16_ts(tO, tPlo + kk * 8, db, idO, 1u);
+        }
+        umma_commit(o_done);
+        umma_commit(&empty[j & 1]);
+      }
+      umma_commit(drain);
+      mbar_wait_bounded(drain, 0, kPfWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;                 // tensor-memory lanes 32*quarter ..
+    const int r = quarter * 32 + lane;            // this thread's row
+    const int t = r / G, g = r - (r / G) * G;
+    const bool row_ok = r < rows_q && tok0 + t < C;
+    const int pos = row_ok ? Lc - C + tok0 + t : pos_max;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = __all_sync(0xffffffffu, pf_wait(&s_full[j & 1], (j >> 1) & 1, abort));
+      if (!ok) break;
+      tc_fence_after();
+      // pass 1: the row maximum of this tile (log2 units, masked)
+      const uint32_t sj = tS + lane_addr + (j & 1) * kPfKeys;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
+        uint32_t v[32];
+        tmem_load32(sj + c4 * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (j * kPfKeys + c4 * 32 + i <= pos) mt = fmaxf(mt, __uint_as_float(v[i]) * sl2);
+      }
+      const float m_new = fmaxf(m, mt);
+      const float alpha = exp2f(m - m_new);
+      m = m_new;
+      // O and the P columns are free once the previous P.V is done
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, pf_wait(o_done, (j - 1) & 1, abort));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t o[32];
+            tmem_load32(tO + lane_addr + c4 * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_store32(tO + lane_addr + c4 * 32, o);
+          }
+        }
+      }
+      // pass 2: weights -> tensor memory (hi, and lo for bf16), row sum
+      float rs = 0.f;
+#pragma unroll
+      for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
+        uint32_t v[32];
+        tmem_load32(sj + c4 * 32, v);
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k0 = j * kPfKeys + c4 * 32 + 2 * i;
+          const float p0 = k0 <= pos ? exp2f(__uint_as_float(v[2 * i]) * sl2 - m_new) : 0.f;
+          const float p1 = k0 + 1 <= pos ? exp2f(__uint_as_float(v[2 * i + 1]) * sl2 - m_new) : 0.f;
+          if (PfPack<T>::kSplit) {
+            PfPack<T>::split2(p0, p1, &hi[i], &lo[i]);
+            rs += p0 + p1;
+          } else {
+            hi[i] = PfPack<T>::round2(p0, p1, &rs);
+          }
+        }
+        tmem_store16(tP + lane_addr + c4 * 16, hi);
+        if (PfPack<T>::kSplit) tmem_store16(tPlo + lane_addr + c4 * 16, lo);
+      }
+      l = l * alpha + rs;
+      if (j == n_tiles - 1) {
+        // keys past pos_max are masked for every row; their V rows may hold
+        // stale or poisoned bits, and 0 * NaN would reach O: zero them
+        const int z0 = pos_max + 1 - j * kPfKeys;
+        if (z0 < kPfKeys) {
+          ok = __all_sync(0xffffffffu, pf_wait(&full[j & 1], (j >> 1) & 1, abort));
+          if (!ok) break;
+          const int tid = threadIdx.x - 64;
+          uint8_t *v0 = sV + (j & 1) * L::KV_BYTES;
+          for (int i = tid; i < NCH * (kPfKeys - z0) * 8; i += 128) {
+            const int c = i / ((kPfKeys - z0) * 8), rem = i % ((kPfKeys - z0) * 8);
+            *reinterpret_cast<uint4 *>(v0 + c * kPfKeys * 128 + (z0 + rem / 8) * 128 +
+                                       (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, pf_wait(o_done, (n_tiles - 1) & 1, abort));
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      float *dst = p.out + ((size_t)(q0 + tok0 + t) * p.num_q_heads + kh * G + g) * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t o[32];
+        tmem_load32(tO + lane_addr + c4 * 32, o);
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4 *>(dst + c4 * 32 + i) =
+                make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                            __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kPfTmemCols);
+  }
+}
+
+}  // namespace pa

@@ -86,3 +86,22 @@ def test_no_oracle_on_the_product_path():
             if f.endswith((".py", ".cu", ".cuh", ".cpp", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.replace("no oracle", ""), f
+
+
+def test_prefill_host_argument_checks(pa):
+    """pa_paged_prefill_attention refuses bad shapes on the host, and an empty
+    call is a no-op, before any CUDA call."""
+    L = pa.lib()
+    nul = None
+
+    def pf(kv=8, seqs=4, toks=16, qh=32, hd=128, bs=16, maxb=4, mq=4, nblk=10, dt=1):
+        return L.pa_paged_prefill_attention(nul, nul, nul, nul, nul, nul, nul, 1.0, kv, seqs,
+                                            toks, qh, hd, bs, maxb, mq, nblk, dt, nul)
+    assert pf(qh=30) == -1              # q heads not a multiple of kv heads
+    assert pf(hd=96) == -2              # unsupported head_dim
+    assert pf(bs=8) == -2               # unsupported block size
+    assert pf(kv=1, qh=32) == -2        # group of 32 > 16
+    assert pf(dt=2) == -1               # fp32 cache
+    assert pf(toks=-1) == -1
+    assert pf(seqs=0) == 0 and pf(toks=0) == 0 and pf(mq=0) == 0
+    assert pf() == -1                   # null pointers
