@@ -8,6 +8,7 @@ of every sequence through the block tables.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa8b]
     python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+    python bench.py --workload prefill       # chunked prefill (tensor cores), TFLOP/s
 
 Prints one JSON line (rank 0).  `value` is the decode attention's algorithmic
 HBM bytes (every K/V element of every cached token read once, plus the block
@@ -45,7 +46,10 @@ WORKLOADS = {
     "long": "long-context paged decode: 8 seqs, 64 q / 8 kv heads, head_dim 128, block 16, bf16, "
             "context lengths uniform 16384..32768, peaked softmax",
     "long32": "long-context paged decode, block 32",
+    "prefill": "chunked prefill: 16 seqs, 512-token chunks on 0..3584 cached tokens, 32 q / 8 kv "
+               "heads, head_dim 128, block 16, bf16 KV, shuffled blocks",
 }
+PREFILL_METRIC = "chunked prefill attention achieved TFLOP/s (% of measured bf16 tensor peak)"
 METRIC = "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_attention_gqa8b.md")
 KERNEL_SOURCES = ["paged_kv_cache_414_b200/csrc/decode_attention.cuh",
@@ -89,6 +93,14 @@ def profiled_traffic(bytes_per_launch: float):
     if not m_sha or not m_tr or not m_alg or m_sha.group(1) != kernel_source_sha():
         return None
     return round(float(m_tr.group(1)) * bytes_per_launch / float(m_alg.group(1)))
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def measured_hbm_peak():
@@ -504,6 +516,331 @@ def run_e2e(pa, wl, K, Wm, dev, world, reduce_max, reduce_sum):
                       "three buffer sets"}
 
 
+# ----------------------------------------------------------------------------- chunked prefill
+
+class PrefillBench:
+    """The chunked-prefill batch (16 sequences, 512-token chunks on top of
+    0..3584 cached tokens, GQA 8B heads, bf16) with the block manager's
+    output for it: each sequence's earlier context allocated, then its chunk
+    appended token by token."""
+
+    def __init__(self, pa, device, rank: int):
+        self.shape = W.SHAPES["gqa8b"]
+        seed = W.SEEDS["gqa8b"] + 100 + 1000 * rank
+        lens, chunks = W.prefill_lens(np.random.default_rng(seed))
+        self.batch = W.make_prefill_batch(self.shape, lens, chunks, seed, device=device)
+        b = self.batch
+        bm = pa.BlockManager(b.num_blocks, self.shape.block_size, b.free_order)
+        slots = []
+        for s in range(b.num_seqs):
+            L, C = int(lens[s]), int(chunks[s])
+            bm.allocate(s, L - C)
+            sl, _ = bm.append_slots([s] * C)
+            slots.append(sl)
+        tables, ctx = bm.block_tables(np.arange(b.num_seqs), b.block_tables.shape[1])
+        bm.close()
+        assert np.array_equal(tables, b.block_tables) and np.array_equal(ctx, b.context_lens)
+        self.slots = np.concatenate(slots).astype(np.int64)
+        self.flops = pa.prefill_flops(lens, chunks, self.shape.num_q_heads, self.shape.head_dim)
+        self.max_query_len = int(chunks.max())
+
+
+def run_prefill_b200(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_414_b200 import build as pbuild
+    pbuild.build()
+    import paged_kv_cache_414_b200 as pa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    K, Wm = args.steps, args.warmup
+    pb = PrefillBench(pa, dev, rank)
+    b, sh = pb.batch, pb.shape
+    T = b.num_tokens
+    d_slots = torch.as_tensor(pb.slots, device=dev)
+    d_tables = torch.as_tensor(b.block_tables, device=dev)
+    d_lens = torch.as_tensor(b.context_lens, device=dev)
+    d_qs = torch.as_tensor(b.query_start, device=dev)
+    out = torch.empty(T, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def step(k=None):
+        # the chunk's cache write, then its attention over the paged context
+        pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, d_slots)
+        if k is not None:
+            ev_a[k].record(stream)
+        pa.pa_paged_prefill_attention(out, b.q, b.k_cache, b.v_cache, d_tables, d_lens, d_qs,
+                                      b.scale, sh.num_kv_heads, pb.max_query_len)
+        if k is not None:
+            ev_b[k].record(stream)
+
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize()
+    pa.pa_device_error(clear=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(K):
+        step(k)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    flags = pa.pa_device_error()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = float(np.mean([ev_a[k].elapsed_time(ev_b[k]) for k in range(K)]))
+
+    def reduce_max(x):
+        return rank_reduce(x, "max", world, dev)
+
+    def reduce_sum(x):
+        return rank_reduce(x, "sum", world, dev)
+
+    ms_max = reduce_max(ms_total)
+    flops_all = reduce_sum(float(pb.flops) * K)
+    value = flops_all / (ms_max * 1e-3) / 1e12
+    achieved = pb.flops / (attn_ms * 1e-3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_prefill_e2e(pa, pb, K, Wm, dev, world, reduce_max, reduce_sum)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = prefill_cpu_baseline(pb, args.cpu_seconds)
+    if rank == 0:
+        line = {
+            "metric": PREFILL_METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": Wm,
+            "ms_per_step": round(ms_max / K, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": sh.dtype,
+            "data": "synthetic",
+            "config": {
+                "workload": f"prefill: {WORKLOADS['prefill']}",
+                "num_seqs_per_gpu": b.num_seqs,
+                "num_tokens_per_step": T,
+                "num_q_heads": sh.num_q_heads,
+                "num_kv_heads": sh.num_kv_heads,
+                "head_dim": sh.head_dim,
+                "block_size": sh.block_size,
+                "mean_context_len": float(np.mean(b.context_lens)),
+                "parallelism": f"dp{world} (independent batches, no collective on the data path)",
+                "l2": "inputs larger than L2 (%.0f MB of K/V pool, %.0f MB of q, %.0f MB of "
+                      "output per step), no flush" % (
+                          2 * b.k_cache.numel() * 2 / 1e6, b.q.numel() * 2 / 1e6,
+                          out.numel() * 4 / 1e6),
+                "step": "reshape_and_cache of the chunk (slots prepared ahead by the host block "
+                        "manager) -> pa_paged_prefill_attention",
+            },
+            "pct_of_measured_bf16_peak": round(100.0 * value / peak / world, 2),
+            "roofline": {
+                "bound": "tensor",
+                "kernel": "paged_prefill_kernel (tcgen05: S = Q K^T, O += P V, P in TMEM)",
+                "achieved": round(achieved, 2),
+                "peak": peak,
+                "peak_source": (f"{peak_kind} bf16_tflops burst (MEASURED_PEAKS.json)"
+                                if peak_kind == "measured" else "fallback 1590 TFLOP/s"),
+                "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": None,
+                "flops_per_launch": pb.flops,
+                "flops_note": "algorithmic: 4*D*Hq*(p+1) per chunk token; the kernel also "
+                              "multiplies the masked half of diagonal tiles and, for bf16, "
+                              "P.V twice (hi + lo weights), which are not counted",
+                "avg_launch_ms": round(attn_ms, 5),
+                "launch_timing": "CUDA events around every prefill call",
+            },
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": 2 * K,
+            "device_error_flags": flags,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_prefill_e2e(pa, pb, K, Wm, dev, world, reduce_max, reduce_sum):
+    """The prefill step through the public API from pinned host buffers: per
+    step the chunk's q, new K/V, slots, block tables, context lengths and
+    query offsets go host -> device as one packed copy, the two kernels run,
+    the fp32 output comes back.  Upload, compute and download run on three
+    streams with two buffer sets, so one step's download overlaps the next
+    step's upload and kernels."""
+    import torch
+    import torch.distributed as dist
+    b, sh = pb.batch, pb.shape
+    T, S = b.num_tokens, b.num_seqs
+    parts = [("q", b.q.dtype, tuple(b.q.shape), 2), ("k", b.k_new.dtype, tuple(b.k_new.shape), 2),
+             ("v", b.v_new.dtype, tuple(b.v_new.shape), 2), ("slots", torch.int64, (T,), 8),
+             ("tables", torch.int32, tuple(b.block_tables.shape), 4),
+             ("lens", torch.int32, (S,), 4), ("qs", torch.int32, (S + 1,), 4)]
+    off, pos = {}, 0
+    for name, _, shape, es in parts:
+        off[name] = pos
+        pos += (int(np.prod(shape)) * es + 255) // 256 * 256
+    total = pos
+
+    def views(buf):
+        return {name: buf[off[name]:off[name] + int(np.prod(shape)) * es].view(dt).view(shape)
+                for name, dt, shape, es in parts}
+
+    NBUF = 2
+    h_buf = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(NBUF)]
+    d_buf = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(NBUF)]
+    h_in, d_in = [views(x) for x in h_buf], [views(x) for x in d_buf]
+    for hv in h_in:
+        hv["q"].copy_(b.q.cpu()); hv["k"].copy_(b.k_new.cpu()); hv["v"].copy_(b.v_new.cpu())
+        hv["slots"].copy_(torch.from_numpy(pb.slots))
+        hv["tables"].copy_(torch.from_numpy(b.block_tables))
+        hv["lens"].copy_(torch.from_numpy(b.context_lens))
+        hv["qs"].copy_(torch.from_numpy(b.query_start))
+    h_out = [torch.empty(T, sh.num_q_heads, sh.head_dim).pin_memory() for _ in range(NBUF)]
+    d_out = [torch.empty(T, sh.num_q_heads, sh.head_dim, device=dev) for _ in range(NBUF)]
+    s_up, s_cmp, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(NBUF)]
+    ev_cmp = [torch.cuda.Event() for _ in range(NBUF)]
+    ev_dn = [torch.cuda.Event() for _ in range(NBUF)]
+    used = [False] * NBUF
+
+    def one(i):
+        j = i % NBUF
+        dv = d_in[j]
+        with torch.cuda.stream(s_up):
+            if used[j]:
+                s_up.wait_event(ev_cmp[j])
+            d_buf[j].copy_(h_buf[j], non_blocking=True)
+            ev_up[j].record(s_up)
+        s_cmp.wait_event(ev_up[j])
+        if used[j]:
+            s_cmp.wait_event(ev_dn[j])
+        pa.pa_reshape_and_cache(dv["k"], dv["v"], b.k_cache, b.v_cache, dv["slots"],
+                                stream=s_cmp)
+        pa.pa_paged_prefill_attention(d_out[j], dv["q"], b.k_cache, b.v_cache, dv["tables"],
+                                      dv["lens"], dv["qs"], b.scale, sh.num_kv_heads,
+                                      pb.max_query_len, stream=s_cmp)
+        ev_cmp[j].record(s_cmp)
+        with torch.cuda.stream(s_dn):
+            s_dn.wait_event(ev_cmp[j])
+            h_out[j].copy_(d_out[j], non_blocking=True)
+            ev_dn[j].record(s_dn)
+        used[j] = True
+
+    for i in range(Wm):
+        one(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(Wm, Wm + K):
+        one(i)
+    torch.cuda.synchronize()
+    dt = reduce_max(time.perf_counter() - t0)
+    flops_all = reduce_sum(float(pb.flops) * K)
+    return {"value": round(flops_all / dt / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(total), "d2h_bytes_per_step": int(h_out[0].numel() * 4),
+            "ms_per_step": round(dt * 1e3 / K, 4),
+            "timing": "host wall clock, synchronize on both sides, max over ranks; one packed "
+                      "upload, two kernels, one download per step on three streams, two buffer "
+                      "sets (PCIe-bound: the step moves its q and fp32 output)"}
+
+
+def prefill_oracle_sample(pb, seqs, kb, vb):
+    """The oracle's chunked prefill for some sequences on the pool bits after
+    the chunk's cache write.  Returns (seconds, flops)."""
+    from oracle import attention as OA
+    b, sh = pb.batch, pb.shape
+    t0 = time.perf_counter()
+    OA.paged_prefill_attention(W.bits(b.q), kb, vb, b.block_tables, b.context_lens,
+                               b.query_start, b.scale, sh.num_kv_heads, sh.block_size, sh.dtype,
+                               seqs=seqs)
+    dt = time.perf_counter() - t0
+    from paged_kv_cache_414_b200 import prefill_flops
+    return dt, prefill_flops(b.context_lens[seqs], b.chunk_lens[seqs], sh.num_q_heads,
+                             sh.head_dim)
+
+
+def prefill_oracle_pool(pb):
+    from oracle import cache_ops as OC
+    b = pb.batch
+    kb, vb = W.bits(b.k_cache), W.bits(b.v_cache)
+    OC.reshape_and_cache(W.bits(b.k_new), W.bits(b.v_new), kb, vb, pb.slots, pb.shape.block_size)
+    return kb, vb
+
+
+def prefill_cpu_baseline(pb, seconds: float):
+    """The oracle on whole sequences of the prefill batch until about
+    `seconds` of CPU work are spent (shortest contexts first)."""
+    kb, vb = prefill_oracle_pool(pb)
+    order = np.argsort(pb.batch.context_lens).tolist()
+    spent, flops, done = 0.0, 0, 0
+    for s in order:
+        dt, f = prefill_oracle_sample(pb, [int(s)], kb, vb)
+        spent += dt
+        flops += f
+        done += 1
+        if spent >= seconds:
+            break
+    return {"value": round(flops / spent / 1e12, 6), "unit": "TFLOP/s",
+            "cores": cpu_cores_used(), "kind": "oracle",
+            "sample": f"{done} of {pb.batch.num_seqs} sequences of the prefill batch (fp64 "
+                      f"attention of every chunk token), {spent:.1f} s of CPU work"}
+
+
+def run_prefill_reference(args, rank, world):
+    """The reference arm for the prefill workload: the CPU oracle."""
+    if rank != 0:
+        return
+    import paged_kv_cache_414_b200 as pa
+    from paged_kv_cache_414_b200 import build as pbuild
+    pbuild.build()
+    K, Wm = args.steps, args.warmup
+    pb = PrefillBench(pa, "cpu", 0)
+    kb, vb = prefill_oracle_pool(pb)
+    order = np.argsort(pb.batch.context_lens).tolist()
+    times, flops = [], []
+    for i in range(Wm + K):
+        dt, f = prefill_oracle_sample(pb, [int(order[i % len(order)])], kb, vb)
+        if i >= Wm:
+            times.append(dt)
+            flops.append(f)
+    value = sum(flops) / sum(times) / 1e12
+    sh = pb.shape
+    line = {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": round(1e3 * sum(times) / K, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"prefill: {WORKLOADS['prefill']}",
+                   "num_seqs_per_gpu": pb.batch.num_seqs, "num_q_heads": sh.num_q_heads,
+                   "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
+                   "block_size": sh.block_size, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores_used(),
+                         "kind": "oracle",
+                         "sample": "one sequence of the prefill batch per step (fp64 attention "
+                                   "of every chunk token)"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- oracle (CPU)
 
 def oracle_step_sample(wl, step: int, seqs):
@@ -617,7 +954,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        if args.workload == "prefill":
+            run_prefill_reference(args, rank, world)
+        else:
+            run_reference(args, rank, world)
         return
     if world > 1:
         import datetime
@@ -628,7 +968,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_b200(args, rank, world, local_rank)
+        if args.workload == "prefill":
+            run_prefill_b200(args, rank, world, local_rank)
+        else:
+            run_b200(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

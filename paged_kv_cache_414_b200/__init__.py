@@ -505,3 +505,14 @@ def decode_bytes(context_lens, num_kv_heads: int, head_dim: int, block_size: int
         L = int(L)
         total += 2 * L * num_kv_heads * head_dim * elem_bytes + 4 * math.ceil(L / block_size)
     return total
+
+
+def prefill_flops(context_lens, chunk_lens, num_q_heads: int, head_dim: int) -> int:
+    """Algorithmic FLOPs of one chunked-prefill attention call: a chunk token
+    at position p costs 2*head_dim*(p+1) for its scores and as much for P.V,
+    per query head; positions run L-C .. L-1, so a sequence contributes
+    4*D*Hq * C*(2L - C + 1)/2."""
+    total = 0
+    for L, C in zip(np.asarray(context_lens).tolist(), np.asarray(chunk_lens).tolist()):
+        total += 4 * head_dim * num_q_heads * (int(C) * (2 * int(L) - int(C) + 1) // 2)
+    return total

@@ -17,7 +17,9 @@
 // in tiles of 128 positions (8 blocks of 16 or 4 of 32), fetched by TMA
 // straight from their physical blocks into 128-byte-swizzled shared memory.
 //
-//   warp 0      TMA producer: Q once, then K/V tiles into a two-stage ring.
+//   warp 0      TMA producer: Q once, then K/V tiles into a three-stage ring;
+//               each lane issues one copy of a tile (one block, one 64-column
+//               chunk, K or V), and K and V land on separate barriers.
 //   warp 1      owns the tensor memory; one lane issues the MMAs:
 //                 S_j = Q K_j^T    (M 128, N 128 keys, K = head_dim), into one
 //                                  of two S buffers, so S_{j+1} runs while the
@@ -32,9 +34,13 @@
 //               tensor memory when the row maximum moves; the epilogue writes
 //               out = O / l.
 //
-// Tensor memory (512 columns): S buffers at 0 and 128, O at 256 (head_dim
-// columns), P_hi at 384 and P_lo at 448 (64 columns each: 128 16-bit
-// weights per row, two per column).
+// Tensor memory: S buffers at columns 0 and 128, O at 256 (head_dim
+// columns).  P_j replaces S_j in its own buffer, 32 keys at a time: the 32
+// columns holding those keys' scores take their 16 columns of hi weights
+// (two per column) and, for bf16, 16 of lo weights.  The MMA that next
+// writes the buffer, S_{j+2}, is issued after P_j . V_j, and MMAs run in
+// issue order.  So the softmax of tile j overlaps P_{j-1} . V_{j-1} and
+// waits for it only before handing P_j over.
 //
 // Every wait is bounded: on time-out a shared abort flag stops every role,
 // PA_DEVERR_TIMEOUT is set, copies and MMAs in flight are waited for (again
@@ -63,6 +69,7 @@ constexpr int kPfKeys = 128;      // keys per K/V tile
 constexpr int kPfThreads = 192;   // producer warp, MMA warp, 4 softmax warps
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint64_t kPfWaitLimitNs = 2000000000ull;
+constexpr int kPfStages = 3;      // K/V ring depth
 
 template <int D>
 struct PrefillSmem {
@@ -71,10 +78,10 @@ struct PrefillSmem {
   static constexpr int Q_BYTES = NCH * REGION;
   static constexpr int KV_BYTES = NCH * kPfKeys * 128;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;       // two stages
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // two stages
-  static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
-  static constexpr int BYTES = OFF_BAR + 128 + 1024;  // barriers + alignment slack
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + kPfStages * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + kPfStages * KV_BYTES;
+  static constexpr int BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
 };
 
 // Bounded wait that also gives up when another role has aborted.
@@ -90,6 +97,14 @@ __device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, volatile
       return false;
     }
   }
+}
+
+// 2^x by the hardware approximation (ex2.approx, flush-to-zero); its error is
+// far below the rounding the weights then get.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Rounding of the softmax weights to the MMA's input type.
@@ -144,15 +159,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t *sK = smem + L::OFF_K;
   uint8_t *sV = smem + L::OFF_V;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
-  uint64_t *full = bars + 0;       // [2] K/V stage landed
-  uint64_t *empty = bars + 2;      // [2] K/V stage consumed
-  uint64_t *q_full = bars + 4;     // Q landed
-  uint64_t *s_full = bars + 5;     // [2] S buffer written
-  uint64_t *p_full = bars + 7;     // P written and O rescaled (128 arrivals)
-  uint64_t *o_done = bars + 8;     // O += P V done
-  uint64_t *drain = bars + 9;      // every MMA done (before freeing tensor memory)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
-  volatile int *abort = reinterpret_cast<volatile int *>(bars + 11);
+  uint64_t *full_k = bars + 0;     // [stages] K tile landed
+  uint64_t *full_v = bars + 3;     // [stages] V tile landed
+  uint64_t *empty = bars + 6;      // [stages] K/V stage consumed
+  uint64_t *q_full = bars + 9;     // Q landed
+  uint64_t *s_full = bars + 10;    // [2] S buffer written
+  uint64_t *p_full = bars + 12;    // P written and O rescaled (128 arrivals)
+  uint64_t *o_done = bars + 13;    // O += P V done
+  uint64_t *drain = bars + 14;     // every MMA done (before freeing tensor memory)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
+  volatile int *abort = reinterpret_cast<volatile int *>(bars + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.x % p.num_seqs;
@@ -177,11 +193,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int rows_q = p.tq * G;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&full[i], 1);
+    for (int i = 0; i < kPfStages; ++i) {
+      mbar_init(&full_k[i], 1);
+      mbar_init(&full_v[i], 1);
       mbar_init(&empty[i], 1);
-      mbar_init(&s_full[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(q_full, 1);
     mbar_init(p_full, 128);
     mbar_init(o_done, 1);
@@ -205,11 +222,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 2 * kPfKeys, tP = tmem + 3 * kPfKeys,
-                 tPlo = tP + kPfKeys / 2;
+  const uint32_t tS = tmem, tO = tmem + 2 * kPfKeys;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // lane -> (block of the tile, 64-column chunk, K or V): BPT * NCH * 2 <= 32 copies
+    constexpr int NCOPY = BPT * NCH * 2;
+    const int cb = lane / (NCH * 2), cc = (lane >> 1) % NCH, ckv = lane & 1;
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
@@ -217,45 +236,44 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_arrive_expect_tx(q_full, NCH * 128 * rows_q);
       for (int c = 0; c < NCH; ++c)
         tma_load_3d(sQ + c * L::REGION, &qmap, c * 64, kh * G, q0 + tok0, q_full);
-      const int32_t *table = p.block_tables + (size_t)s * p.max_blocks;
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !pf_wait(&empty[st], ((j >> 1) - 1) & 1, abort)) break;
-        const int b0 = j * BPT;
-        const int nb = min(BPT, nb_used - b0);
-        int ids[BPT];
-        int nvalid = 0;
-#pragma unroll
-        for (int b = 0; b < BPT; ++b) {
-          ids[b] = -1;
-          if (b < nb) {
-            const int id = __ldg(table + b0 + b);
-            if (id >= 0 && id < p.num_blocks) {
-              ids[b] = id;
-              ++nvalid;
-            } else {
-              flag_error(PA_DEVERR_BLOCK_ID);
-            }
-          }
-        }
-        mbar_arrive_expect_tx(&full[st], nvalid * 2 * NCH * B * 128);
-#pragma unroll
-        for (int b = 0; b < BPT; ++b) {
-          if (ids[b] < 0) continue;
-          const int row = (ids[b] * p.num_kv_heads + kh) * B;
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            const int off = st * L::KV_BYTES + c * kPfKeys * 128 + b * B * 128;
-            tma_load_2d(sK + off, &kmap, c * 64, row, &full[st]);
-            tma_load_2d(sV + off, &vmap, c * 64, row, &full[st]);
-          }
-        }
-        issued = j + 1;
+    }
+    const int32_t *table = p.block_tables + (size_t)s * p.max_blocks;
+    int issued = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j % kPfStages;
+      // this lane's block id, fetched before the stage is free
+      const int b0 = j * BPT;
+      int id = -1;
+      bool bad = false;
+      if (lane < NCOPY && cb < nb_used - b0) {
+        const int v = __ldg(table + b0 + cb);
+        if (v >= 0 && v < p.num_blocks) id = v; else bad = true;
       }
-      // copies still in flight must land before the CTA exits
-      for (int j = max(0, issued - 2); j < issued; ++j)
-        mbar_wait_bounded(&full[j & 1], (j >> 1) & 1, kPfWaitLimitNs);
+      if (bad && cc == 0 && ckv == 0) flag_error(PA_DEVERR_BLOCK_ID);
+      if (j >= kPfStages) {
+        const bool w = lane == 0 ? pf_wait(&empty[st], (j / kPfStages - 1) & 1, abort) : true;
+        if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      }
+      const unsigned valid = __ballot_sync(0xffffffffu, id >= 0);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full_k[st], __popc(valid & 0x55555555u) * B * 128);
+        mbar_arrive_expect_tx(&full_v[st], __popc(valid & 0xAAAAAAAAu) * B * 128);
+      }
+      __syncwarp();
+      if (id >= 0) {
+        const int off = st * L::KV_BYTES + cc * kPfKeys * 128 + cb * B * 128;
+        const int row = (id * p.num_kv_heads + kh) * B;
+        if (ckv == 0) tma_load_2d(sK + off, &kmap, cc * 64, row, &full_k[st]);
+        else tma_load_2d(sV + off, &vmap, cc * 64, row, &full_v[st]);
+      }
+      issued = j + 1;
+    }
+    // copies still in flight must land before the CTA exits
+    if (lane == 0) {
+      for (int j = max(0, issued - kPfStages); j < issued; ++j) {
+        mbar_wait_bounded(&full_k[j % kPfStages], (j / kPfStages) & 1, kPfWaitLimitNs);
+        mbar_wait_bounded(&full_v[j % kPfStages], (j / kPfStages) & 1, kPfWaitLimitNs);
+      }
       mbar_wait_bounded(q_full, 0, kPfWaitLimitNs);
     }
   } else if (warp == 1) {
@@ -266,7 +284,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint32_t idO = umma_idesc_f16(kBf, kPfRows, D, false, true);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
       auto issue_s = [&](int j) {
-        const uint32_t k0 = aK + (j & 1) * L::KV_BYTES;
+        const uint32_t k0 = aK + (j % kPfStages) * L::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kPfKeys * 128) + (kk & 3) * 32;
@@ -276,29 +294,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         umma_commit(&s_full[j & 1]);
       };
-      bool ok = pf_wait(q_full, 0, abort) && pf_wait(&full[0], 0, abort);
+      bool ok = pf_wait(q_full, 0, abort) && pf_wait(&full_k[0], 0, abort);
       if (ok) {
         tc_fence_after();
         issue_s(0);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         if (j + 1 < n_tiles) {
-          if (!pf_wait(&full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort)) break;
+          if (!pf_wait(&full_k[(j + 1) % kPfStages], ((j + 1) / kPfStages) & 1, abort)) break;
           tc_fence_after();
           issue_s(j + 1);
         }
         if (!pf_wait(p_full, j & 1, abort)) break;
+        if (!pf_wait(&full_v[j % kPfStages], (j / kPfStages) & 1, abort)) break;
         tc_fence_after();
-        const uint32_t v0 = aV + (j & 1) * L::KV_BYTES;
+        const uint32_t v0 = aV + (j % kPfStages) * L::KV_BYTES;
+        const uint32_t pj = tS + (j & 1) * kPfKeys;
 #pragma unroll
         for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-          // 16 keys: 8 columns of P, 16 rows of V
+          // 16 keys: 8 columns of P (hi at 32*(kk/2) + 8*(kk%2), lo 16 further), 16 rows of V
           const uint64_t db = umma_desc_sw128(v0 + kk * 16 * 128, kPfKeys * 128, 1024);
-          umma_f16_ts(tO, tP + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
-          if (PfPack<T>::kSplit) umma_f16_ts(tO, tPlo + kk * 8, db, idO, 1u);
+          const uint32_t pc = pj + (kk >> 1) * 32 + (kk & 1) * 8;
+          umma_f16_ts(tO, pc, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          if (PfPack<T>::kSplit) umma_f16_ts(tO, pc + 16, db, idO, 1u);
         }
         umma_commit(o_done);
-        umma_commit(&empty[j & 1]);
+        umma_commit(&empty[j % kPfStages]);
       }
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, kPfWaitLimitNs);
@@ -310,35 +331,89 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int t = r / G, g = r - (r / G) * G;
     const bool row_ok = r < rows_q && tok0 + t < C;
     const int pos = row_ok ? Lc - C + tok0 + t : pos_max;
+    const int pos_min = Lc - C + tok0;              // the first chunk token's position
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
+    const bool pos_scale = sl2 > 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = __all_sync(0xffffffffu, pf_wait(&s_full[j & 1], (j >> 1) & 1, abort));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: the row maximum of this tile (log2 units, masked)
+      // pass 1: the row maximum of the raw scores (masked on diagonal tiles)
       const uint32_t sj = tS + lane_addr + (j & 1) * kPfKeys;
-      float mt = -INFINITY;
+      const bool diag = (j + 1) * kPfKeys - 1 > pos_min;   // some key past some row's position
+      float mx[8];
 #pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll 1
       for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
         uint32_t v[32];
         tmem_load32(sj + c4 * 32, v);
+        const int kbase = j * kPfKeys + c4 * 32;
+        if (!pos_scale) {           // general scale: maximum of the scaled scores
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (j * kPfKeys + c4 * 32 + i <= pos) mt = fmaxf(mt, __uint_as_float(v[i]) * sl2);
+          for (int i = 0; i < 32; ++i)
+            if (kbase + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]) * sl2);
+        } else if (diag) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (kbase + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+        }
       }
-      const float m_new = fmaxf(m, mt);
-      const float alpha = exp2f(m - m_new);
+      // with a positive scale the maximum of the raw scores, scaled once
+      const float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mt = pos_scale ? mr * sl2 : mr;
+      // Lazy rescaling: the reference maximum m moves only when the tile's
+      // maximum exceeds it by more than 8 (log2 units), so weights stay below
+      // 2^8 and O is rescaled in tensor memory only on those rare steps.
+      const bool bump = mt > m + 8.f;
+      const float m_new = bump ? mt : m;
+      const float alpha = bump ? fast_exp2(m - m_new) : 1.f;
       m = m_new;
-      // O and the P columns are free once the previous P.V is done
+      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, row sum
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
+        uint32_t v[32];
+        tmem_load32(sj + c4 * 32, v);
+        const int kbase = j * kPfKeys + c4 * 32;
+        float pr[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pr[i] = fast_exp2(fmaf(__uint_as_float(v[i]), sl2, -m_new));
+        if (diag) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pr[i] = kbase + i <= pos ? pr[i] : 0.f;
+        }
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (PfPack<T>::kSplit) {
+            PfPack<T>::split2(pr[2 * i], pr[2 * i + 1], &hi[i], &lo[i]);
+            sum[i & 3] += pr[2 * i] + pr[2 * i + 1];
+          } else {
+            hi[i] = PfPack<T>::round2(pr[2 * i], pr[2 * i + 1], &sum[i & 3]);
+          }
+        }
+        // the 32 score columns just read take these keys' weights
+        tmem_store16(sj + c4 * 32, hi);
+        if (PfPack<T>::kSplit) tmem_store16(sj + c4 * 32 + 16, lo);
+      }
+      const float rs = (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      l = l * alpha + rs;
+      // O is stable once the previous P.V is done; rescale it if the
+      // reference maximum moved
       if (j > 0) {
         ok = __all_sync(0xffffffffu, pf_wait(o_done, (j - 1) & 1, abort));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+        if (__any_sync(0xffffffffu, bump)) {
+#pragma unroll 1
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t o[32];
             tmem_load32(tO + lane_addr + c4 * 32, o);
@@ -348,38 +423,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
-      // pass 2: weights -> tensor memory (hi, and lo for bf16), row sum
-      float rs = 0.f;
-#pragma unroll
-      for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
-        uint32_t v[32];
-        tmem_load32(sj + c4 * 32, v);
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k0 = j * kPfKeys + c4 * 32 + 2 * i;
-          const float p0 = k0 <= pos ? exp2f(__uint_as_float(v[2 * i]) * sl2 - m_new) : 0.f;
-          const float p1 = k0 + 1 <= pos ? exp2f(__uint_as_float(v[2 * i + 1]) * sl2 - m_new) : 0.f;
-          if (PfPack<T>::kSplit) {
-            PfPack<T>::split2(p0, p1, &hi[i], &lo[i]);
-            rs += p0 + p1;
-          } else {
-            hi[i] = PfPack<T>::round2(p0, p1, &rs);
-          }
-        }
-        tmem_store16(tP + lane_addr + c4 * 16, hi);
-        if (PfPack<T>::kSplit) tmem_store16(tPlo + lane_addr + c4 * 16, lo);
-      }
-      l = l * alpha + rs;
       if (j == n_tiles - 1) {
         // keys past pos_max are masked for every row; their V rows may hold
         // stale or poisoned bits, and 0 * NaN would reach O: zero them
         const int z0 = pos_max + 1 - j * kPfKeys;
         if (z0 < kPfKeys) {
-          ok = __all_sync(0xffffffffu, pf_wait(&full[j & 1], (j >> 1) & 1, abort));
+          ok = __all_sync(0xffffffffu,
+                          pf_wait(&full_v[j % kPfStages], (j / kPfStages) & 1, abort));
           if (!ok) break;
           const int tid = threadIdx.x - 64;
-          uint8_t *v0 = sV + (j & 1) * L::KV_BYTES;
+          uint8_t *v0 = sV + (j % kPfStages) * L::KV_BYTES;
           for (int i = tid; i < NCH * (kPfKeys - z0) * 8; i += 128) {
             const int c = i / ((kPfKeys - z0) * 8), rem = i % ((kPfKeys - z0) * 8);
             *reinterpret_cast<uint4 *>(v0 + c * kPfKeys * 128 + (z0 + rem / 8) * 128 +

@@ -149,3 +149,17 @@ def test_bad_chunk_reports_instead_of_faulting(pa, cuda_device):
     assert pa.pa_device_error() & pa.DEVERR["context_len"]
     o = out.cpu().numpy()
     assert (o[:4] == 7.0).all() and np.isfinite(o[4:]).all() and not (o[4:] == 7.0).all()
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.06, 0.9])
+def test_any_scale(pa, cuda_device, scale):
+    """The softmax scale is any float: zero (uniform weights), negative, and
+    large enough that the lazy rescaling of O triggers often."""
+    sh = W.Shape(16, 4, 128, 16, "bf16")
+    b = W.make_prefill_batch(sh, [300, 77, 1000], [300, 20, 129], seed=31, device=cuda_device,
+                             poison="nan")
+    b.scale = scale
+    got, want = run_prefill(pa, b)
+    assert np.isfinite(got).all()
+    assert max_abs_err(got, want) <= TOL
+    assert pa.pa_device_error() == 0
