@@ -25,8 +25,13 @@
 //                                  of two S buffers, so S_{j+1} runs while the
 //                                  softmax works on S_j;
 //                 O  += P_j V_j    (M 128, N = head_dim, K 128 keys).
-//   warps 2-5   softmax, one thread per row (tensor-memory lane): online
-//               maximum and sum in fp32; P_j goes to tensor memory, where the
+//   warps 2-9   softmax, two threads per row: warps w and w+4 share the
+//               tensor-memory lanes of one row quarter and take 64 keys each;
+//               they exchange partial maxima every tile (through spare
+//               tensor-memory columns, ordered by a 64-arrival mbarrier per
+//               pair, waited on with the same bounded wait as everything else)
+//               and their partial sums once at the end.  Online maximum and sum
+//               in fp32; P_j goes to tensor memory, where the
 //               P.V MMA reads it as its A operand.  For bf16, P = P_hi + P_lo
 //               (both bf16, two MMAs), so P carries about 2^-17 relative
 //               rounding instead of bf16's 2^-9; for fp16 one fp16 P whose
@@ -35,7 +40,7 @@
 //               out = O / l.
 //
 // Tensor memory: S buffers at columns 0 and 128, O at 256 (head_dim
-// columns).  P_j replaces S_j in its own buffer, 32 keys at a time: the 32
+// columns), exchange columns from 384.  P_j replaces S_j in its own buffer, 32 keys at a time: the 32
 // columns holding those keys' scores take their 16 columns of hi weights
 // (two per column) and, for bf16, 16 of lo weights.  The MMA that next
 // writes the buffer, S_{j+2}, is issued after P_j . V_j, and MMAs run in
@@ -66,7 +71,7 @@ struct PrefillParams {
 
 constexpr int kPfRows = 128;      // query rows per CTA
 constexpr int kPfKeys = 128;      // keys per K/V tile
-constexpr int kPfThreads = 192;   // producer warp, MMA warp, 4 softmax warps
+constexpr int kPfThreads = 320;   // producer warp, MMA warp, 8 softmax warps
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint64_t kPfWaitLimitNs = 2000000000ull;
 constexpr int kPfStages = 3;      // K/V ring depth
@@ -164,11 +169,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t *empty = bars + 6;      // [stages] K/V stage consumed
   uint64_t *q_full = bars + 9;     // Q landed
   uint64_t *s_full = bars + 10;    // [2] S buffer written
-  uint64_t *p_full = bars + 12;    // P written and O rescaled (128 arrivals)
+  uint64_t *p_full = bars + 12;    // P written and O rescaled (256 arrivals)
   uint64_t *o_done = bars + 13;    // O += P V done
   uint64_t *drain = bars + 14;     // every MMA done (before freeing tensor memory)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
-  volatile int *abort = reinterpret_cast<volatile int *>(bars + 16);
+  uint64_t *pair = bars + 15;      // [4] the two softmax threads of each row quarter
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
+  volatile int *abort = reinterpret_cast<volatile int *>(bars + 20);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.x % p.num_seqs;
@@ -200,7 +206,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(q_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
+    for (int i = 0; i < 4; ++i) mbar_init(&pair[i], 64);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort = 0;
@@ -327,12 +334,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;                 // tensor-memory lanes 32*quarter ..
+    const int half = (warp - 2) >> 2;             // keys 64*half .. 64*half+63 of a tile
     const int r = quarter * 32 + lane;            // this thread's row
     const int t = r / G, g = r - (r / G) * G;
     const bool row_ok = r < rows_q && tok0 + t < C;
     const int pos = row_ok ? Lc - C + tok0 + t : pos_max;
     const int pos_min = Lc - C + tok0;              // the first chunk token's position
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tX = tmem + lane_addr + 3 * kPfKeys;   // exchange columns
     const float sl2 = p.scale_log2;
     const bool pos_scale = sl2 > 0.f;
     float m = -INFINITY, l = 0.f;
@@ -341,17 +350,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       ok = __all_sync(0xffffffffu, pf_wait(&s_full[j & 1], (j >> 1) & 1, abort));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: the row maximum of the raw scores (masked on diagonal tiles)
-      const uint32_t sj = tS + lane_addr + (j & 1) * kPfKeys;
-      const bool diag = (j + 1) * kPfKeys - 1 > pos_min;   // some key past some row's position
+      // pass 1: this half's maximum of the raw scores (masked on diagonal tiles)
+      const uint32_t sj = tS + lane_addr + (j & 1) * kPfKeys + half * 64;
+      const int kh0 = j * kPfKeys + half * 64;   // first key of this half
+      const bool diag = kh0 + 63 > pos_min;      // some key past some row's position
       float mx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll 1
-      for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
+      for (int c4 = 0; c4 < 2; ++c4) {
         uint32_t v[32];
         tmem_load32(sj + c4 * 32, v);
-        const int kbase = j * kPfKeys + c4 * 32;
+        const int kbase = kh0 + c4 * 32;
         if (!pos_scale) {           // general scale: maximum of the scaled scores
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -365,24 +375,35 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
         }
       }
+      float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      // the row's maximum: exchange with the other half (column per half,
+      // two sets by tile parity, so a partner still reading this tile's
+      // value is never overwritten by the next tile's)
+      tmem_store1(tX + 2 * (j & 1) + half, __float_as_uint(mr));
+      tc_fence_before();
+      mbar_arrive(&pair[quarter]);
+      ok = __all_sync(0xffffffffu, pf_wait(&pair[quarter], j & 1, abort));
+      if (!ok) break;
+      tc_fence_after();
+      mr = fmaxf(mr, __uint_as_float(tmem_load1(tX + 2 * (j & 1) + (1 - half))));
       // with a positive scale the maximum of the raw scores, scaled once
-      const float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mt = pos_scale ? mr * sl2 : mr;
       // Lazy rescaling: the reference maximum m moves only when the tile's
       // maximum exceeds it by more than 8 (log2 units), so weights stay below
-      // 2^8 and O is rescaled in tensor memory only on those rare steps.
+      // 2^8 and O is rescaled in tensor memory only on those rare steps.  Both
+      // halves of a row take the same decisions.
       const bool bump = mt > m + 8.f;
       const float m_new = bump ? mt : m;
       const float alpha = bump ? fast_exp2(m - m_new) : 1.f;
       m = m_new;
-      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, row sum
+      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, partial row sum
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-      for (int c4 = 0; c4 < kPfKeys / 32; ++c4) {
+      for (int c4 = 0; c4 < 2; ++c4) {
         uint32_t v[32];
         tmem_load32(sj + c4 * 32, v);
-        const int kbase = j * kPfKeys + c4 * 32;
+        const int kbase = kh0 + c4 * 32;
         float pr[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pr[i] = fast_exp2(fmaf(__uint_as_float(v[i]), sl2, -m_new));
@@ -404,22 +425,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_store16(sj + c4 * 32, hi);
         if (PfPack<T>::kSplit) tmem_store16(sj + c4 * 32 + 16, lo);
       }
-      const float rs = (sum[0] + sum[1]) + (sum[2] + sum[3]);
-      l = l * alpha + rs;
-      // O is stable once the previous P.V is done; rescale it if the
-      // reference maximum moved
+      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      // O is stable once the previous P.V is done; rescale this half's
+      // columns if the reference maximum moved
       if (j > 0) {
         ok = __all_sync(0xffffffffu, pf_wait(o_done, (j - 1) & 1, abort));
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, bump)) {
 #pragma unroll 1
-          for (int c4 = 0; c4 < D / 32; ++c4) {
+          for (int c4 = 0; c4 < D / 64; ++c4) {
             uint32_t o[32];
-            tmem_load32(tO + lane_addr + c4 * 32, o);
+            const uint32_t oc = tO + lane_addr + half * (D / 2) + c4 * 32;
+            tmem_load32(oc, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_store32(tO + lane_addr + c4 * 32, o);
+            tmem_store32(oc, o);
           }
         }
       }
@@ -433,7 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (!ok) break;
           const int tid = threadIdx.x - 64;
           uint8_t *v0 = sV + (j % kPfStages) * L::KV_BYTES;
-          for (int i = tid; i < NCH * (kPfKeys - z0) * 8; i += 128) {
+          for (int i = tid; i < NCH * (kPfKeys - z0) * 8; i += 256) {
             const int c = i / ((kPfKeys - z0) * 8), rem = i % ((kPfKeys - z0) * 8);
             *reinterpret_cast<uint4 *>(v0 + c * kPfKeys * 128 + (z0 + rem / 8) * 128 +
                                        (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
@@ -446,13 +467,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     if (ok) ok = __all_sync(0xffffffffu, pf_wait(o_done, (n_tiles - 1) & 1, abort));
     if (ok) {
+      // the row sum: this half's plus the other half's (one more pair phase)
+      tmem_store1(tX + 4 + half, __float_as_uint(l));
+      tc_fence_before();
+      mbar_arrive(&pair[quarter]);
+      ok = __all_sync(0xffffffffu, pf_wait(&pair[quarter], n_tiles & 1, abort));
+    }
+    if (ok) {
       tc_fence_after();
+      l += __uint_as_float(tmem_load1(tX + 4 + (1 - half)));
       const float inv = 1.f / l;
-      float *dst = p.out + ((size_t)(q0 + tok0 + t) * p.num_q_heads + kh * G + g) * D;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
+      float *dst = p.out + ((size_t)(q0 + tok0 + t) * p.num_q_heads + kh * G + g) * D +
+                   half * (D / 2);
+#pragma unroll 1
+      for (int c4 = 0; c4 < D / 64; ++c4) {
         uint32_t o[32];
-        tmem_load32(tO + lane_addr + c4 * 32, o);
+        tmem_load32(tO + lane_addr + half * (D / 2) + c4 * 32, o);
         if (row_ok) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4)

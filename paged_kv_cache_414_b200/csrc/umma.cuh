@@ -143,6 +143,25 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
+// One 32-bit TMEM column of this thread's lane <-> a register (with the wait).
+__device__ __forceinline__ uint32_t tmem_load1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r)
+      : "r"(taddr)
+      : "memory");
+  return r;
+}
+__device__ __forceinline__ void tmem_store1(uint32_t taddr, uint32_t r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r)
+      : "memory");
+}
+
 // Registers -> 16 consecutive TMEM columns of this thread's lane, and wait.
 __device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
