@@ -322,7 +322,7 @@ int launch_prefill(const PrefillArgs &a, int dev) {
   p.max_blocks = a.max_blocks;
   p.num_blocks = a.num_blocks;
   p.tq = tq;
-  p.q_tiles = (a.max_query_len + tq - 1) / tq;
+  p.q_tiles = (a.max_query_len + 2 * tq - 1) / (2 * tq);   // a CTA takes two query tiles
   const long long nx = (long long)p.q_tiles * a.num_seqs;
   if (nx >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
   cudaLaunchConfig_t cfg = {};

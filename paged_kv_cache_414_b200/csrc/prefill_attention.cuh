@@ -11,41 +11,43 @@
 // causally to positions 0 .. L_s - C_s + i:
 //   out[t, h] = softmax(scale * q[t, h] . K_s[0..p]) V_s[0..p].
 //
-// Work split: one CTA per (sequence, kv head, query tile).  A query tile is
-// 128 rows = TQ = 128 / G chunk tokens x the G query heads that share the kv
-// head, so every K/V tile fetched from the pool serves all 128 rows.  Keys go
-// in tiles of 128 positions (8 blocks of 16 or 4 of 32), fetched by TMA
-// straight from their physical blocks into 128-byte-swizzled shared memory.
+// Work split: one CTA per (sequence, kv head, pair of query tiles).  A query
+// tile is 128 rows = TQ = 128 / G chunk tokens x the G query heads that share
+// the kv head; the CTA's two tiles (A, then B: 2 TQ consecutive tokens) share
+// every K/V tile fetched from the pool.  Keys go in tiles of 128 positions
+// (8 blocks of 16 or 4 of 32), fetched by TMA straight from their physical
+// blocks into 128-byte-swizzled shared memory.
 //
-//   warp 0      TMA producer: Q once, then K/V tiles into a three-stage ring;
+//   warp 0      TMA producer: both Q tiles once, then K/V tiles into a ring;
 //               each lane issues one copy of a tile (one block, one 64-column
 //               chunk, K or V), and K and V land on separate barriers.
-//   warp 1      owns the tensor memory; one lane issues the MMAs:
-//                 S_j = Q K_j^T    (M 128, N 128 keys, K = head_dim), into one
-//                                  of two S buffers, so S_{j+1} runs while the
-//                                  softmax works on S_j;
-//                 O  += P_j V_j    (M 128, N = head_dim, K 128 keys).
-//   warps 2-9   softmax, two threads per row: warps w and w+4 share the
-//               tensor-memory lanes of one row quarter and take 64 keys each;
-//               they exchange partial maxima every tile (through spare
-//               tensor-memory columns, ordered by a 64-arrival mbarrier per
-//               pair, waited on with the same bounded wait as everything else)
-//               and their partial sums once at the end.  Online maximum and sum
-//               in fp32; P_j goes to tensor memory, where the
-//               P.V MMA reads it as its A operand.  For bf16, P = P_hi + P_lo
-//               (both bf16, two MMAs), so P carries about 2^-17 relative
-//               rounding instead of bf16's 2^-9; for fp16 one fp16 P whose
-//               rounded weights are also what the sum adds.  O is rescaled in
-//               tensor memory when the row maximum moves; the epilogue writes
+//   warp 1      owns the tensor memory; one lane issues the MMAs, alternating
+//               between the query tiles so that one tile's MMAs run while the
+//               other tile's softmax does:
+//                 S_X = Q_X K_j^T   (M 128, N 128 keys, K = head_dim)
+//                 O_X += P_X V_j    (M 128, N = head_dim, K 128 keys)
+//               in the order S_A(0) S_B(0), then per tile j: O_A += P_A V_j,
+//               S_A(j+1), O_B += P_B V_j, S_B(j+1).
+//   warps 2-9   softmax of tile A, warps 10-17 of tile B, two threads per
+//               row: warps w and w+4 share the tensor-memory lanes of one row
+//               quarter and take 64 keys each, exchanging partial maxima every
+//               tile (through shared memory, ordered by a 64-arrival mbarrier
+//               per pair and the same bounded wait as everything else) and
+//               partial sums once at the end.  Online maximum and sum in
+//               fp32; the weights go to tensor memory, where the P.V MMA reads
+//               them as its A operand.  For bf16, P = P_hi + P_lo (both bf16, two
+//               MMAs), so P carries about 2^-17 relative rounding instead of
+//               bf16's 2^-9; for fp16 one fp16 P whose rounded weights are
+//               also what the sum adds.  O is rescaled in tensor memory when
+//               the row maximum moves by more than 2^8; the epilogue writes
 //               out = O / l.
 //
-// Tensor memory: S buffers at columns 0 and 128, O at 256 (head_dim
-// columns), exchange columns from 384.  P_j replaces S_j in its own buffer, 32 keys at a time: the 32
-// columns holding those keys' scores take their 16 columns of hi weights
-// (two per column) and, for bf16, 16 of lo weights.  The MMA that next
-// writes the buffer, S_{j+2}, is issued after P_j . V_j, and MMAs run in
-// issue order.  So the softmax of tile j overlaps P_{j-1} . V_{j-1} and
-// waits for it only before handing P_j over.
+// Tensor memory (512 columns): tile A's S at 0 and O at 128, tile B's S at
+// 256 and O at 384.  P replaces S in its own columns, 16 keys at a time: the
+// 16 columns holding those keys' scores take their 8 columns of hi weights
+// (two per column) and, for bf16, 8 of lo weights.  The MMA that next writes
+// a tile's S columns is issued after that tile's P.V, and MMAs run in issue
+// order.
 //
 // Every wait is bounded: on time-out a shared abort flag stops every role,
 // PA_DEVERR_TIMEOUT is set, copies and MMAs in flight are waited for (again
@@ -65,28 +67,29 @@ struct PrefillParams {
   const int32_t *query_start;    // [S + 1]
   float scale_log2;              // scale * log2(e)
   int num_seqs, num_tokens, num_q_heads, num_kv_heads, group, max_blocks, num_blocks;
-  int q_tiles;                   // query tiles per sequence in the grid
+  int q_tiles;                   // CTAs (pairs of query tiles) per sequence in the grid
   int tq;                        // chunk tokens per query tile (128 / group)
 };
 
-constexpr int kPfRows = 128;      // query rows per CTA
+constexpr int kPfRows = 128;      // query rows per query tile
 constexpr int kPfKeys = 128;      // keys per K/V tile
-constexpr int kPfThreads = 320;   // producer warp, MMA warp, 8 softmax warps
+constexpr int kPfThreads = 576;   // producer warp, MMA warp, 2 x 8 softmax warps
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint64_t kPfWaitLimitNs = 2000000000ull;
-constexpr int kPfStages = 3;      // K/V ring depth
 
 template <int D>
 struct PrefillSmem {
   static constexpr int NCH = D / 64;                  // 64-column chunks of a row
+  static constexpr int STAGES = D == 128 ? 2 : 3;     // K/V ring depth
   static constexpr int REGION = kPfRows * 128;        // one 64-column chunk of 128 rows
-  static constexpr int Q_BYTES = NCH * REGION;
+  static constexpr int Q_TILE = NCH * REGION;         // one query tile
   static constexpr int KV_BYTES = NCH * kPfKeys * 128;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + kPfStages * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + kPfStages * KV_BYTES;
-  static constexpr int BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+  static constexpr int OFF_Q = 0;                     // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_X = OFF_BAR + 256;         // pair exchange: [tile][set][half][row]
+  static constexpr int BYTES = OFF_X + 2 * 3 * 2 * 128 * 4 + 1024;  // + alignment slack
 };
 
 // Bounded wait that also gives up when another role has aborted.
@@ -156,6 +159,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                          const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
   using L = PrefillSmem<D>;
   constexpr int NCH = L::NCH;
+  constexpr int NST = L::STAGES;
   constexpr int BPT = kPfKeys / B;                    // blocks per K/V tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -164,17 +168,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t *sK = smem + L::OFF_K;
   uint8_t *sV = smem + L::OFF_V;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
-  uint64_t *full_k = bars + 0;     // [stages] K tile landed
-  uint64_t *full_v = bars + 3;     // [stages] V tile landed
-  uint64_t *empty = bars + 6;      // [stages] K/V stage consumed
-  uint64_t *q_full = bars + 9;     // Q landed
-  uint64_t *s_full = bars + 10;    // [2] S buffer written
-  uint64_t *p_full = bars + 12;    // P written and O rescaled (256 arrivals)
-  uint64_t *o_done = bars + 13;    // O += P V done
-  uint64_t *drain = bars + 14;     // every MMA done (before freeing tensor memory)
-  uint64_t *pair = bars + 15;      // [4] the two softmax threads of each row quarter
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
-  volatile int *abort = reinterpret_cast<volatile int *>(bars + 20);
+  uint64_t *full_k = bars + 0;     // [NST] K tile landed
+  uint64_t *full_v = bars + 3;     // [NST] V tile landed
+  uint64_t *empty = bars + 6;      // [NST] K/V stage consumed by all four MMAs
+  uint64_t *q_full = bars + 9;     // both Q tiles landed
+  uint64_t *s_full = bars + 10;    // [query tile] S written
+  uint64_t *p_full = bars + 12;    // [query tile] P written, O rescaled (256 arrivals)
+  uint64_t *o_done = bars + 14;    // [query tile] O += P V done
+  uint64_t *drain = bars + 16;     // every MMA done (before freeing tensor memory)
+  uint64_t *pair = bars + 17;      // [query tile][row quarter] the two threads of a row
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
+  volatile int *abort = reinterpret_cast<volatile int *>(bars + 26);
+  float *xch = reinterpret_cast<float *>(smem + L::OFF_X);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.x % p.num_seqs;
@@ -186,29 +191,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int q0 = __ldg(p.query_start + s);
   const int C = __ldg(p.query_start + s + 1) - q0;
   const int Lc = __ldg(p.context_lens + s);
-  const int tok0 = qt * p.tq;
+  const int tok0 = qt * 2 * p.tq;
   if (C < 0 || C > Lc || Lc > p.max_blocks * B || q0 < 0 || q0 + C > p.num_tokens) {
     if (threadIdx.x == 0 && kh == 0 && qt == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
     return;
   }
   if (tok0 >= C) return;                               // uniform over the CTA
-  const int ntok = min(p.tq, C - tok0);
+  const int ntok = min(2 * p.tq, C - tok0);
   const int pos_max = Lc - C + tok0 + ntok - 1;        // last position any row sees
   const int n_tiles = pos_max / kPfKeys + 1;
   const int nb_used = pos_max / B + 1;                 // blocks holding positions 0..pos_max
   const int rows_q = p.tq * G;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPfStages; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&full_k[i], 1);
       mbar_init(&full_v[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(q_full, 1);
-    mbar_init(p_full, 256);
-    for (int i = 0; i < 4; ++i) mbar_init(&pair[i], 64);
-    mbar_init(o_done, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 256);
+      for (int q = 0; q < 4; ++q) mbar_init(&pair[x * 4 + q], 64);
+      mbar_init(&o_done[x], 1);
+    }
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -218,10 +225,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tmem_relinquish();
   }
   if (rows_q < kPfRows) {     // Q rows no chunk token fills: zeros, not stale bits
-    for (int i = threadIdx.x; i < NCH * (kPfRows - rows_q) * 8; i += kPfThreads) {
-      const int c = i / ((kPfRows - rows_q) * 8), rem = i % ((kPfRows - rows_q) * 8);
-      *reinterpret_cast<uint4 *>(sQ + c * L::REGION + (rows_q + rem / 8) * 128 + (rem % 8) * 16) =
-          make_uint4(0, 0, 0, 0);
+    const int per_tile = NCH * (kPfRows - rows_q) * 8;
+    for (int i = threadIdx.x; i < 2 * per_tile; i += kPfThreads) {
+      const int x = i / per_tile, rem0 = i % per_tile;
+      const int c = rem0 / ((kPfRows - rows_q) * 8), rem = rem0 % ((kPfRows - rows_q) * 8);
+      *reinterpret_cast<uint4 *>(sQ + x * L::Q_TILE + c * L::REGION + (rows_q + rem / 8) * 128 +
+                                 (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
   }
@@ -229,7 +238,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 2 * kPfKeys;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -240,14 +248,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
-      mbar_arrive_expect_tx(q_full, NCH * 128 * rows_q);
-      for (int c = 0; c < NCH; ++c)
+      // tile B past the chunk: load tile A's tokens again (finite, never stored)
+      const int zb = tok0 + p.tq < C ? q0 + tok0 + p.tq : q0 + tok0;
+      mbar_arrive_expect_tx(q_full, 2 * NCH * 128 * rows_q);
+      for (int c = 0; c < NCH; ++c) {
         tma_load_3d(sQ + c * L::REGION, &qmap, c * 64, kh * G, q0 + tok0, q_full);
+        tma_load_3d(sQ + L::Q_TILE + c * L::REGION, &qmap, c * 64, kh * G, zb, q_full);
+      }
     }
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks;
     int issued = 0;
     for (int j = 0; j < n_tiles; ++j) {
-      const int st = j % kPfStages;
+      const int st = j % NST;
       // this lane's block id, fetched before the stage is free
       const int b0 = j * BPT;
       int id = -1;
@@ -257,8 +269,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (v >= 0 && v < p.num_blocks) id = v; else bad = true;
       }
       if (bad && cc == 0 && ckv == 0) flag_error(PA_DEVERR_BLOCK_ID);
-      if (j >= kPfStages) {
-        const bool w = lane == 0 ? pf_wait(&empty[st], (j / kPfStages - 1) & 1, abort) : true;
+      if (j >= NST) {
+        const bool w = lane == 0 ? pf_wait(&empty[st], (j / NST - 1) & 1, abort) : true;
         if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
       const unsigned valid = __ballot_sync(0xffffffffu, id >= 0);
@@ -277,9 +289,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     // copies still in flight must land before the CTA exits
     if (lane == 0) {
-      for (int j = max(0, issued - kPfStages); j < issued; ++j) {
-        mbar_wait_bounded(&full_k[j % kPfStages], (j / kPfStages) & 1, kPfWaitLimitNs);
-        mbar_wait_bounded(&full_v[j % kPfStages], (j / kPfStages) & 1, kPfWaitLimitNs);
+      for (int j = max(0, issued - NST); j < issued; ++j) {
+        mbar_wait_bounded(&full_k[j % NST], (j / NST) & 1, kPfWaitLimitNs);
+        mbar_wait_bounded(&full_v[j % NST], (j / NST) & 1, kPfWaitLimitNs);
       }
       mbar_wait_bounded(q_full, 0, kPfWaitLimitNs);
     }
@@ -290,103 +302,114 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint32_t idS = umma_idesc_f16(kBf, kPfRows, kPfKeys, false, false);
       const uint32_t idO = umma_idesc_f16(kBf, kPfRows, D, false, true);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
-      auto issue_s = [&](int j) {
-        const uint32_t k0 = aK + (j % kPfStages) * L::KV_BYTES;
+      auto issue_s = [&](int x, int j) {        // S_x = Q_x K_j^T
+        const uint32_t q = aQ + x * L::Q_TILE, k0 = aK + (j % NST) * L::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kPfKeys * 128) + (kk & 3) * 32;
-          const uint64_t da = umma_desc_sw128(aQ + (kk >> 2) * L::REGION + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = umma_desc_sw128(k0 + off, 16, 1024);
-          umma_f16_ss(tS + (j & 1) * kPfKeys, da, db, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * L::REGION + (kk & 3) * 32;
+          umma_f16_ss(tmem + x * 256, umma_desc_sw128(q + off, 16, 1024),
+                      umma_desc_sw128(k0 + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[j & 1]);
+        umma_commit(&s_full[x]);
+      };
+      auto issue_pv = [&](int x, int j) {       // O_x += P_x V_j
+        const uint32_t v0 = aV + (j % NST) * L::KV_BYTES, pj = tmem + x * 256;
+#pragma unroll
+        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
+          // 16 keys: their 16 score columns hold 8 columns of hi weights, then
+          // (bf16) 8 of lo weights; 16 rows of V
+          const uint64_t db = umma_desc_sw128(v0 + kk * 16 * 128, kPfKeys * 128, 1024);
+          const uint32_t pc = pj + kk * 16;
+          umma_f16_ts(tmem + x * 256 + 128, pc, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          if (PfPack<T>::kSplit) umma_f16_ts(tmem + x * 256 + 128, pc + 8, db, idO, 1u);
+        }
+        umma_commit(&o_done[x]);
       };
       bool ok = pf_wait(q_full, 0, abort) && pf_wait(&full_k[0], 0, abort);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles) {
-          if (!pf_wait(&full_k[(j + 1) % kPfStages], ((j + 1) / kPfStages) & 1, abort)) break;
-          tc_fence_after();
-          issue_s(j + 1);
-        }
-        if (!pf_wait(p_full, j & 1, abort)) break;
-        if (!pf_wait(&full_v[j % kPfStages], (j / kPfStages) & 1, abort)) break;
+        // tile A: its P.V, then its next S (which overwrites its P, in issue order)
+        if (!pf_wait(&p_full[0], j & 1, abort)) break;
+        if (!pf_wait(&full_v[j % NST], (j / NST) & 1, abort)) break;
         tc_fence_after();
-        const uint32_t v0 = aV + (j % kPfStages) * L::KV_BYTES;
-        const uint32_t pj = tS + (j & 1) * kPfKeys;
-#pragma unroll
-        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-          // 16 keys: 8 columns of P (hi at 32*(kk/2) + 8*(kk%2), lo 16 further), 16 rows of V
-          const uint64_t db = umma_desc_sw128(v0 + kk * 16 * 128, kPfKeys * 128, 1024);
-          const uint32_t pc = pj + (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_f16_ts(tO, pc, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
-          if (PfPack<T>::kSplit) umma_f16_ts(tO, pc + 16, db, idO, 1u);
+        issue_pv(0, j);
+        const bool more = j + 1 < n_tiles;
+        if (more) {
+          if (!pf_wait(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1, abort)) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
         }
-        umma_commit(o_done);
-        umma_commit(&empty[j % kPfStages]);
+        // tile B
+        if (!pf_wait(&p_full[1], j & 1, abort)) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(&empty[j % NST]);
+        if (more) issue_s(1, j + 1);
       }
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, kPfWaitLimitNs);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    const int x = (warp - 2) >> 3;                // query tile: warps 2-9 A, 10-17 B
+    const int half = ((warp - 2) >> 2) & 1;       // keys 64*half .. 64*half+63 of a tile
     const int quarter = warp & 3;                 // tensor-memory lanes 32*quarter ..
-    const int half = (warp - 2) >> 2;             // keys 64*half .. 64*half+63 of a tile
-    const int r = quarter * 32 + lane;            // this thread's row
+    const int r = quarter * 32 + lane;            // this thread's row of the tile
     const int t = r / G, g = r - (r / G) * G;
-    const bool row_ok = r < rows_q && tok0 + t < C;
-    const int pos = row_ok ? Lc - C + tok0 + t : pos_max;
-    const int pos_min = Lc - C + tok0;              // the first chunk token's position
+    const int tokx = tok0 + x * p.tq;             // the tile's first chunk token
+    const bool row_ok = r < rows_q && tokx + t < C;
+    const int pos = row_ok ? Lc - C + tokx + t : pos_max;
+    const int pos_min = min(Lc - C + tokx, pos_max);
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tX = tmem + lane_addr + 3 * kPfKeys;   // exchange columns
+    const uint32_t tSx = tmem + x * 256 + lane_addr, tOx = tSx + 128;
+    uint64_t *pr_bar = &pair[x * 4 + quarter];
+    // exchange slots: [tile][set: tile parity 0/1, 2 = row sums][half][row]
+    auto slot = [&](int set, int hf) { return xch + ((x * 3 + set) * 2 + hf) * 128 + r; };
     const float sl2 = p.scale_log2;
     const bool pos_scale = sl2 > 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      ok = __all_sync(0xffffffffu, pf_wait(&s_full[j & 1], (j >> 1) & 1, abort));
+      ok = __all_sync(0xffffffffu, pf_wait(&s_full[x], j & 1, abort));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: this half's maximum of the raw scores (masked on diagonal tiles)
-      const uint32_t sj = tS + lane_addr + (j & 1) * kPfKeys + half * 64;
+      // this half's 64 scores, read once (two loads) and kept in registers
+      const uint32_t sj = tSx + half * 64;
       const int kh0 = j * kPfKeys + half * 64;   // first key of this half
       const bool diag = kh0 + 63 > pos_min;      // some key past some row's position
+      uint32_t v[64];
+      tmem_load32(sj, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_load32(sj + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      // pass 1: the maximum of the raw scores (masked on diagonal tiles)
       float mx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-#pragma unroll 1
-      for (int c4 = 0; c4 < 2; ++c4) {
-        uint32_t v[32];
-        tmem_load32(sj + c4 * 32, v);
-        const int kbase = kh0 + c4 * 32;
-        if (!pos_scale) {           // general scale: maximum of the scaled scores
+      if (!pos_scale) {             // general scale: maximum of the scaled scores
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (kbase + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]) * sl2);
-        } else if (diag) {
+        for (int i = 0; i < 64; ++i)
+          if (kh0 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]) * sl2);
+      } else if (diag) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (kbase + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
-        } else {
+        for (int i = 0; i < 64; ++i)
+          if (kh0 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
-        }
+        for (int i = 0; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
       }
       float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      // the row's maximum: exchange with the other half (column per half,
-      // two sets by tile parity, so a partner still reading this tile's
-      // value is never overwritten by the next tile's)
-      tmem_store1(tX + 2 * (j & 1) + half, __float_as_uint(mr));
-      tc_fence_before();
-      mbar_arrive(&pair[quarter]);
-      ok = __all_sync(0xffffffffu, pf_wait(&pair[quarter], j & 1, abort));
+      // the row's maximum: exchange with the other half (two slot sets by tile
+      // parity, so a partner still reading this tile's value is never
+      // overwritten by the next tile's)
+      *slot(j & 1, half) = mr;
+      mbar_arrive(pr_bar);
+      ok = __all_sync(0xffffffffu, pf_wait(pr_bar, j & 1, abort));
       if (!ok) break;
-      tc_fence_after();
-      mr = fmaxf(mr, __uint_as_float(tmem_load1(tX + 2 * (j & 1) + (1 - half))));
+      mr = fmaxf(mr, *reinterpret_cast<volatile float *>(slot(j & 1, 1 - half)));
       // with a positive scale the maximum of the raw scores, scaled once
       const float mt = pos_scale ? mr * sl2 : mr;
       // Lazy rescaling: the reference maximum m moves only when the tile's
@@ -397,63 +420,66 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const float m_new = bump ? mt : m;
       const float alpha = bump ? fast_exp2(m - m_new) : 1.f;
       m = m_new;
-      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, partial row sum
+      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, partial row
+      // sum; per 16 keys, their 16 score columns take 8 columns of hi weights
+      // and (bf16) 8 of lo weights; one wait for all the stores
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-      for (int c4 = 0; c4 < 2; ++c4) {
-        uint32_t v[32];
-        tmem_load32(sj + c4 * 32, v);
-        const int kbase = kh0 + c4 * 32;
-        float pr[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pr[i] = fast_exp2(fmaf(__uint_as_float(v[i]), sl2, -m_new));
-        if (diag) {
+      for (int c = 0; c < 4; ++c) {
+        uint32_t hi[8], lo[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pr[i] = kbase + i <= pos ? pr[i] : 0.f;
-        }
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 8; ++i) {
+          const int k = c * 16 + 2 * i;
+          float p0 = fast_exp2(fmaf(__uint_as_float(v[k]), sl2, -m_new));
+          float p1 = fast_exp2(fmaf(__uint_as_float(v[k + 1]), sl2, -m_new));
+          if (diag) {
+            p0 = kh0 + k <= pos ? p0 : 0.f;
+            p1 = kh0 + k + 1 <= pos ? p1 : 0.f;
+          }
           if (PfPack<T>::kSplit) {
-            PfPack<T>::split2(pr[2 * i], pr[2 * i + 1], &hi[i], &lo[i]);
-            sum[i & 3] += pr[2 * i] + pr[2 * i + 1];
+            PfPack<T>::split2(p0, p1, &hi[i], &lo[i]);
+            sum[i & 3] += p0 + p1;
           } else {
-            hi[i] = PfPack<T>::round2(pr[2 * i], pr[2 * i + 1], &sum[i & 3]);
+            hi[i] = PfPack<T>::round2(p0, p1, &sum[i & 3]);
           }
         }
-        // the 32 score columns just read take these keys' weights
-        tmem_store16(sj + c4 * 32, hi);
-        if (PfPack<T>::kSplit) tmem_store16(sj + c4 * 32 + 16, lo);
+        tmem_store8_async(sj + c * 16, hi);
+        if (PfPack<T>::kSplit) tmem_store8_async(sj + c * 16 + 8, lo);
       }
+      tmem_store_wait();
       l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
       // O is stable once the previous P.V is done; rescale this half's
       // columns if the reference maximum moved
       if (j > 0) {
-        ok = __all_sync(0xffffffffu, pf_wait(o_done, (j - 1) & 1, abort));
+        ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (j - 1) & 1, abort));
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, bump)) {
 #pragma unroll 1
-          for (int c4 = 0; c4 < D / 64; ++c4) {
-            uint32_t o[32];
-            const uint32_t oc = tO + lane_addr + half * (D / 2) + c4 * 32;
-            tmem_load32(oc, o);
+          for (int c = 0; c < D / 2; c += 16) {        // this half's D/2 columns
+            uint32_t o[16];
+            const uint32_t oc = tOx + half * (D / 2) + c;
+            tmem_load16(oc, o);
+            uint32_t o8[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_store32(oc, o);
+            for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_store8(oc, o8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[8 + i]) * alpha);
+            tmem_store8(oc + 8, o8);
           }
         }
       }
-      if (j == n_tiles - 1) {
+      if (x == 0 && j == n_tiles - 1) {
         // keys past pos_max are masked for every row; their V rows may hold
-        // stale or poisoned bits, and 0 * NaN would reach O: zero them
+        // stale or poisoned bits, and 0 * NaN would reach O: zero them (tile
+        // A's threads; tile B's P.V is issued after tile A's)
         const int z0 = pos_max + 1 - j * kPfKeys;
         if (z0 < kPfKeys) {
-          ok = __all_sync(0xffffffffu,
-                          pf_wait(&full_v[j % kPfStages], (j / kPfStages) & 1, abort));
+          ok = __all_sync(0xffffffffu, pf_wait(&full_v[j % NST], (j / NST) & 1, abort));
           if (!ok) break;
           const int tid = threadIdx.x - 64;
-          uint8_t *v0 = sV + (j % kPfStages) * L::KV_BYTES;
+          uint8_t *v0 = sV + (j % NST) * L::KV_BYTES;
           for (int i = tid; i < NCH * (kPfKeys - z0) * 8; i += 256) {
             const int c = i / ((kPfKeys - z0) * 8), rem = i % ((kPfKeys - z0) * 8);
             *reinterpret_cast<uint4 *>(v0 + c * kPfKeys * 128 + (z0 + rem / 8) * 128 +
@@ -463,30 +489,29 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[x]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, pf_wait(o_done, (n_tiles - 1) & 1, abort));
+    if (ok) ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (n_tiles - 1) & 1, abort));
     if (ok) {
       // the row sum: this half's plus the other half's (one more pair phase)
-      tmem_store1(tX + 4 + half, __float_as_uint(l));
-      tc_fence_before();
-      mbar_arrive(&pair[quarter]);
-      ok = __all_sync(0xffffffffu, pf_wait(&pair[quarter], n_tiles & 1, abort));
+      *slot(2, half) = l;
+      mbar_arrive(pr_bar);
+      ok = __all_sync(0xffffffffu, pf_wait(pr_bar, n_tiles & 1, abort));
     }
     if (ok) {
       tc_fence_after();
-      l += __uint_as_float(tmem_load1(tX + 4 + (1 - half)));
+      l += *reinterpret_cast<volatile float *>(slot(2, 1 - half));
       const float inv = 1.f / l;
-      float *dst = p.out + ((size_t)(q0 + tok0 + t) * p.num_q_heads + kh * G + g) * D +
+      float *dst = p.out + ((size_t)(q0 + tokx + t) * p.num_q_heads + kh * G + g) * D +
                    half * (D / 2);
 #pragma unroll 1
-      for (int c4 = 0; c4 < D / 64; ++c4) {
-        uint32_t o[32];
-        tmem_load32(tO + lane_addr + half * (D / 2) + c4 * 32, o);
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t o[16];
+        tmem_load16(tOx + half * (D / 2) + c4 * 16, o);
         if (row_ok) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4 *>(dst + c4 * 32 + i) =
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4 *>(dst + c4 * 16 + i) =
                 make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
                             __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
         }
