@@ -71,9 +71,15 @@ def parse():
 
 # ----------------------------------------------------------------------------- helpers
 
-def kernel_source_sha() -> str:
+PREFILL_PROFILE = os.path.join(ROOT, "profiles", "prefill_attention_16x512.md")
+PREFILL_SOURCES = ["paged_kv_cache_414_b200/csrc/prefill_attention.cuh",
+                   "paged_kv_cache_414_b200/csrc/umma.cuh",
+                   "paged_kv_cache_414_b200/csrc/pa_device.cuh"]
+
+
+def kernel_source_sha(sources=None) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in (KERNEL_SOURCES if sources is None else sources):
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -93,6 +99,21 @@ def profiled_traffic(bytes_per_launch: float):
     if not m_sha or not m_tr or not m_alg or m_sha.group(1) != kernel_source_sha():
         return None
     return round(float(m_tr.group(1)) * bytes_per_launch / float(m_alg.group(1)))
+
+
+def prefill_profiled_traffic():
+    """DRAM bytes (read + write) of one prefill launch of the bench workload
+    from the committed ncu summary; None unless it was taken on the current
+    kernel source."""
+    try:
+        text = open(PREFILL_PROFILE).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha(PREFILL_SOURCES):
+        return None
+    return int(float(m_tr.group(1)))
 
 
 def measured_tensor_peak():
@@ -659,7 +680,9 @@ def run_prefill_b200(args, rank, world, local_rank):
                                 if peak_kind == "measured" else "fallback 1590 TFLOP/s"),
                 "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": None,
+                "traffic": prefill_profiled_traffic(),
+                "traffic_note": "ncu dram__bytes_read + dram__bytes_write of one launch of this "
+                                "workload (profiles/prefill_attention_16x512.md)",
                 "flops_per_launch": pb.flops,
                 "flops_note": "algorithmic: 4*D*Hq*(p+1) per chunk token; the kernel also "
                               "multiplies the masked half of diagonal tiles and, for bf16, "
