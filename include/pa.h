@@ -246,8 +246,9 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
  *   context_lens int32 [num_seqs] (device), tokens including the chunk
  *   query_start  int32 [num_seqs + 1] (device), non-decreasing, query_start[0] = 0,
  *                query_start[num_seqs] = num_tokens
- *   max_query_len host upper bound of every C_s (sizes the grid; longer chunks
- *                are not computed)
+ *   max_query_len host upper bound of every C_s (sizes the grid; the rows of a
+ *                longer chunk past what the grid covers are not computed, and
+ *                PA_DEVERR_CONTEXT_LEN is set)
  * head_dim 64 or 128, block_size 16 or 32, group size up to 16, fp16 or
  * bf16.  Runs on the tensor cores (tcgen05): P is rounded to the cache dtype
  * before P.V, so the result carries that rounding (relative 2^-9 per weight

@@ -196,6 +196,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (threadIdx.x == 0 && kh == 0 && qt == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
     return;
   }
+  // a chunk longer than the grid covers (max_query_len too small): its last
+  // rows are not computed; say so
+  if (threadIdx.x == 0 && kh == 0 && qt == 0 && C > p.q_tiles * 2 * p.tq)
+    flag_error(PA_DEVERR_CONTEXT_LEN);
   if (tok0 >= C) return;                               // uniform over the CTA
   const int ntok = min(2 * p.tq, C - tok0);
   const int pos_max = Lc - C + tok0 + ntok - 1;        // last position any row sees

@@ -149,6 +149,18 @@ def test_bad_chunk_reports_instead_of_faulting(pa, cuda_device):
     assert pa.pa_device_error() & pa.DEVERR["context_len"]
     o = out.cpu().numpy()
     assert (o[:4] == 7.0).all() and np.isfinite(o[4:]).all() and not (o[4:] == 7.0).all()
+    # max_query_len so small that the grid (two 32-token query tiles per CTA at
+    # G = 4) misses the end of a 100-token chunk: reported, the covered rows
+    # computed, the rest left alone
+    b2 = W.make_prefill_batch(sh, [150], [100], seed=2, device=dev)
+    out2 = torch.full((100, 8, 64), 7.0, device=dev)
+    pa.pa_paged_prefill_attention(out2, b2.q, b2.k_cache, b2.v_cache,
+                                  torch.as_tensor(b2.block_tables, device=dev),
+                                  torch.as_tensor(b2.context_lens, device=dev),
+                                  torch.as_tensor(b2.query_start, device=dev), b2.scale, 2, 10)
+    assert pa.pa_device_error() & pa.DEVERR["context_len"]
+    o2 = out2.cpu().numpy()
+    assert np.isfinite(o2[:64]).all() and not (o2[:64] == 7.0).all() and (o2[64:] == 7.0).all()
 
 
 @pytest.mark.parametrize("scale", [0.0, -0.06, 0.9])
