@@ -46,6 +46,9 @@ WORKLOADS = {
     "long": "long-context paged decode: 8 seqs, 64 q / 8 kv heads, head_dim 128, block 16, bf16, "
             "context lengths uniform 16384..32768, peaked softmax",
     "long32": "long-context paged decode, block 32",
+    "cow": "parallel sampling with copy-on-write: 32 prompts (64..512 tokens) x 8 branches sharing "
+           "the prompt blocks, 32 q / 8 kv heads, head_dim 128, block 16, bf16; the timed steps "
+           "start at the first append (copy_blocks of every shared partial last block)",
     "prefill": "chunked prefill: 16 seqs, 512-token chunks on 0..3584 cached tokens, 32 q / 8 kv "
                "heads, head_dim 128, block 16, bf16 KV, shuffled blocks",
 }
@@ -225,6 +228,10 @@ class Workload:
     def __init__(self, name: str, device, seed_offset: int, steps_total: int):
         import torch
         self.name = name
+        self.cyclic = False
+        if name == "cow":
+            self._init_cow(device, seed_offset, steps_total)
+            return
         sh = W.SHAPES[name]
         self.shape = sh
         seed = rank_seed(name, seed_offset)
@@ -244,16 +251,78 @@ class Workload:
         self.scale = 1.0 / math.sqrt(sh.head_dim)
         self.elem = 2
 
+    def _init_cow(self, device, seed_offset: int, steps_total: int):
+        """32 prompts forked into 8 branches each; the prompts' K/V are written
+        into the pool when the first manager is built.  The step inputs are
+        one seeded draw reused every step (the bytes moved are the same)."""
+        from types import SimpleNamespace
+        sh = W.SHAPES["cow"]
+        self.shape = sh
+        self.cyclic = True          # timed steps replay steps 0.. (copy-on-write first)
+        seed = rank_seed("cow", seed_offset)
+        cw = W.cow_workload(device=device, steps=steps_total, seed=seed)
+        self.cw = cw
+        B = sh.block_size
+        k_cache, v_cache = W.empty_pool(sh, cw.num_blocks, seed, device=device)
+        q, k_new, v_new = cw.step_inputs(0)
+        self.batch = SimpleNamespace(k_cache=k_cache, v_cache=v_cache, q=q, k_new=k_new,
+                                     v_new=v_new, num_blocks=cw.num_blocks,
+                                     free_order=cw.free_order)
+        # context after step 0's append: the prompt plus the branch's first token
+        self.lens0 = np.repeat(cw.prompt_lens.astype(np.int64) + 1, cw.branches)
+        self.maxb = max(math.ceil((int(P) + steps_total) / B) for P in cw.prompt_lens)
+        self.S = cw.num_seqs
+        self.device = device
+        self.scale = 1.0 / math.sqrt(sh.head_dim)
+        self.elem = 2
+        self._prompts_written = False
+
     def bytes_per_step(self, step: int) -> int:
+        """Algorithmic (logical) bytes: every cached token of every sequence;
+        for shared prompt blocks that is once per branch reading them."""
         from paged_kv_cache_414_b200 import decode_bytes
         return decode_bytes(self.lens0 + step, self.shape.num_kv_heads, self.shape.head_dim,
                             self.shape.block_size, self.elem)
 
     def new_manager(self, pa):
+        """A native manager in the state before step 0 (for the cow workload the
+        prompts are allocated and forked, and their K/V written the first time)."""
         bm = pa.BlockManager(self.batch.num_blocks, self.shape.block_size, self.batch.free_order)
-        for s in range(self.S):
-            bm.allocate(s, int(self.lens0[s]) - 1)
+        if self.name != "cow":
+            for s in range(self.S):
+                bm.allocate(s, int(self.lens0[s]) - 1)
+            return bm
+        import torch
+        cw = self.cw
+        slots = []
+        for pr, P in enumerate(cw.prompt_lens):
+            slots.append(bm.allocate(cw.seq_id(pr, 0), int(P)))
+            for br in range(1, cw.branches):
+                bm.fork(cw.seq_id(pr, 0), cw.seq_id(pr, br))
+        if not self._prompts_written:
+            pa.pa_reshape_and_cache(cw.prompt_k, cw.prompt_v, self.batch.k_cache,
+                                    self.batch.v_cache,
+                                    torch.as_tensor(np.concatenate(slots), device=self.device))
+            self._prompts_written = True
         return bm
+
+    def oracle_manager(self, step: int):
+        """The oracle's manager after `step` steps, and the slots of step `step`."""
+        from oracle.block_manager import BlockManager as OracleBM
+        bm = OracleBM(self.batch.num_blocks, self.shape.block_size, self.batch.free_order)
+        if self.name != "cow":
+            for s in range(self.S):
+                bm.allocate(s, int(self.lens0[s]) - 1 + step)
+        else:
+            cw = self.cw
+            for pr, P in enumerate(cw.prompt_lens):
+                bm.allocate(cw.seq_id(pr, 0), int(P))
+                for br in range(1, cw.branches):
+                    bm.fork(cw.seq_id(pr, 0), cw.seq_id(pr, br))
+            for _ in range(step):
+                for s in range(self.S):
+                    bm.append_slot(s)
+        return bm, [bm.append_slot(s)[0] for s in range(self.S)]
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -279,7 +348,13 @@ def run_b200(args, rank, world, local_rank):
     bm = wl.new_manager(pa)
     seqs = np.arange(S)
     d_tables, d_lens, d_pairs = [], [], []
-    for step in range(K + Wm):
+    # step indices: warm-up steps, then the timed ones; a cyclic workload
+    # (copy-on-write) times steps 0.. again after its warm-up, so that the
+    # timed region starts with the copies of the first append
+    nprep = K if wl.cyclic else K + Wm
+    warm_idx = (lambda i: i % K) if wl.cyclic else (lambda i: i)   # noqa: E731
+    timed_idx = (lambda k: k) if wl.cyclic else (lambda k: Wm + k)  # noqa: E731
+    for step in range(nprep):
         slots, pairs = bm.append_slots(seqs)
         tables, lens = bm.block_tables(seqs, wl.maxb)
 
@@ -292,14 +367,21 @@ def run_b200(args, rank, world, local_rank):
     out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
     # kernels launched per timed step: the fused decode step and its split
     # merge, plus copy_blocks on steps with copy-on-write pairs
-    timed_launches = sum(2 + (d_pairs[Wm + k] is not None) for k in range(K))
+    timed_launches = sum(2 + (d_pairs[timed_idx(k)] is not None) for k in range(K))
+    # a pool smaller than twice L2 is flushed (a 256 MB memset) before every
+    # timed step, outside per-step CUDA-event spans that then make the time
+    pool_bytes = 2 * b.k_cache.numel() * b.k_cache.element_size()
+    flush = pool_bytes < 2 * 126 * 2 ** 20
+    flush_buf = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if flush else None
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
 
     # Per-call events only when a step has other kernels (copy-on-write
     # copies) to separate from the decode call: an event recorded between two
     # launches ends the programmatic overlap of the second with the first.
     # Otherwise the decode call is the whole step and its average duration is
     # the timed region over K (launch gaps included, so never optimistic).
-    per_call_events = any(d_pairs[Wm + k] is not None for k in range(K))
+    per_call_events = flush or any(d_pairs[timed_idx(k)] is not None for k in range(K))
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
 
@@ -316,7 +398,7 @@ def run_b200(args, rank, world, local_rank):
             ev_b[timed_idx].record(stream)
 
     for i in range(Wm):
-        step(i)
+        step(warm_idx(i))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -331,7 +413,12 @@ def run_b200(args, rank, world, local_rank):
         dist.barrier()
     t0.record(stream)
     for k in range(K):
-        step(Wm + k, k)
+        if flush:
+            flush_buf.zero_()
+            ev_s[k].record(stream)
+        step(timed_idx(k), k)
+        if flush:
+            ev_e[k].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -339,11 +426,13 @@ def run_b200(args, rank, world, local_rank):
     clk = clocks.stop()
     flags = pa.pa_device_error()
     ms_total = t0.elapsed_time(t1)
+    if flush:   # the steps alone, without the flushes between them
+        ms_total = float(sum(ev_s[k].elapsed_time(ev_e[k]) for k in range(K)))
     if per_call_events:
         attn_ms = [ev_a[k].elapsed_time(ev_b[k]) for k in range(K)]
     else:
         attn_ms = [ms_total / K] * K
-    bytes_steps = [wl.bytes_per_step(Wm + k) for k in range(K)]
+    bytes_steps = [wl.bytes_per_step(timed_idx(k)) for k in range(K)]
     my_bytes = float(sum(bytes_steps))
 
     reduce_max = lambda x: rank_reduce(x, "max", world, dev)   # noqa: E731
@@ -359,7 +448,9 @@ def run_b200(args, rank, world, local_rank):
     bytes_launch = float(np.mean(bytes_steps))
     achieved = bytes_launch / (attn_avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
-    traffic = profiled_traffic(bytes_launch)
+    # the committed ncu summary is of the gqa8b launch; other workloads run
+    # other kernel instances or (shared prefixes) other DRAM/L2 splits
+    traffic = profiled_traffic(bytes_launch) if args.workload == "gqa8b" else None
 
     e2e = None
     if not args.no_e2e:
@@ -390,9 +481,13 @@ def run_b200(args, rank, world, local_rank):
                 "num_kv_heads": sh.num_kv_heads,
                 "head_dim": sh.head_dim,
                 "block_size": B,
-                "mean_context_len": float(np.mean(wl.lens0)) + Wm + (K - 1) / 2,
+                "mean_context_len": float(np.mean(wl.lens0)) + float(np.mean(
+                    [timed_idx(k) for k in range(K)])),
                 "parallelism": f"dp{world} (independent batches, no collective on the data path)",
-                "l2": "inputs larger than L2: %.2f GB of KV read per step, no flush" % (bytes_launch / 1e9),
+                "l2": ("K/V pool %.0f MB, under twice L2: L2 flushed (256 MB memset) before "
+                       "every timed step, outside the per-step CUDA-event spans" % (pool_bytes / 1e6)
+                       if flush else "inputs larger than L2: %.2f GB of KV read per step, no flush"
+                       % (bytes_launch / 1e9)),
                 "step": "host block manager (prepared ahead) -> copy_blocks if any -> pa_decode_step (cache write of the new token + paged decode attention) -> split merge",
             },
             "pct_of_measured_hbm_peak": round(100.0 * value / peak / world, 2),
@@ -871,14 +966,10 @@ def oracle_step_sample(wl, step: int, seqs):
     slots, its own cache write, its own attention.  Returns (out, bytes)."""
     from oracle import attention as OA
     from oracle import cache_ops as OC
-    from oracle.block_manager import BlockManager as OracleBM
     sh = wl.shape
     B = sh.block_size
     b = wl.batch
-    bm = OracleBM(b.num_blocks, B, b.free_order)
-    for s in range(wl.S):
-        bm.allocate(s, int(wl.lens0[s]) - 1 + step)
-    slots = [bm.append_slot(s)[0] for s in range(wl.S)]
+    bm, slots = wl.oracle_manager(step)
     need = sorted({x for s in seqs for x in bm.block_table(s)})
     remap = {x: i for i, x in enumerate(need)}
     import torch
