@@ -175,3 +175,27 @@ def test_any_scale(pa, cuda_device, scale):
     assert np.isfinite(got).all()
     assert max_abs_err(got, want) <= TOL
     assert pa.pa_device_error() == 0
+
+
+def test_bad_block_id_reports_instead_of_faulting(pa, cuda_device):
+    """A block-table entry outside the pool is skipped by the copy engine and
+    reported in the error word; the other sequence's rows still match the
+    oracle."""
+    pa.pa_device_error(clear=True)
+    sh = W.Shape(8, 2, 128, 16, "bf16")
+    b = W.make_prefill_batch(sh, [300, 200], [40, 64], seed=8, device=cuda_device)
+    dev = cuda_device
+    tables = b.block_tables.copy()
+    tables[0, 3] = b.num_blocks + 11                      # sequence 0 only
+    out = torch.empty(b.num_tokens, 8, 128, device=dev)
+    pa.pa_paged_prefill_attention(out, b.q, b.k_cache, b.v_cache,
+                                  torch.as_tensor(tables, device=dev),
+                                  torch.as_tensor(b.context_lens, device=dev),
+                                  torch.as_tensor(b.query_start, device=dev), b.scale, 2, 64)
+    assert pa.pa_device_error() & pa.DEVERR["block_id"]
+    want = OA.paged_prefill_attention(W.bits(b.q), W.bits(b.k_cache), W.bits(b.v_cache),
+                                      b.block_tables, b.context_lens, b.query_start, b.scale, 2,
+                                      16, "bf16", seqs=[1])
+    rows = np.arange(b.query_start[1], b.query_start[2])
+    assert max_abs_err(out.cpu().numpy()[rows], want[rows]) <= TOL
+    assert pa.pa_device_error() == 0
