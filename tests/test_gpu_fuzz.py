@@ -1,9 +1,9 @@
 """Randomized GPU parity sweep: seeded random configurations across the whole
 supported space -- head_dim 64/128, block size 16/32, fp16/bf16, query-head
 groups 1..16, ragged and empty sequences, NaN poison in every unused slot --
-for the two-call decode step, the fused decode step under random launch
-tunings, and chunked prefill, each against the oracle (2e-3 max-abs, the pool
-bit for bit)."""
+for the two-call decode step (a third of the cases under random launch
+tunings), the fused decode step and chunked prefill, each against the oracle
+(2e-3 max-abs, the pool bit for bit)."""
 import numpy as np
 import pytest
 import torch
