@@ -945,7 +945,7 @@ template <int D, int GMW>
 __global__ void __launch_bounds__(128, 6)
     paged_decode_merge_kernel(const DecodeParams p, int w_total, int hc) {
   constexpr int VPL = D / 32;
-  constexpr int UNR = 8 / GMW;   // partials per batch of loads
+  constexpr int UNR = 16 / GMW;   // partials per batch of loads
   using VecT = typename std::conditional<VPL == 4, float4, float2>::type;
   grid_dependency_wait();
   const int lane = threadIdx.x & 31;
