@@ -250,12 +250,13 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
  *                longer chunk past what the grid covers are not computed, and
  *                PA_DEVERR_CONTEXT_LEN is set)
  * head_dim 64 or 128, block_size 16 or 32, group size up to 16, fp16 or
- * bf16.  Runs on the tensor cores (tcgen05): P is rounded to the cache dtype
- * before P.V, so the result carries that rounding (relative 2^-9 per weight
- * for bf16, 2^-12 for fp16) besides the fp32 accumulation.  No workspace,
- * nothing allocated.  A chunk longer than its context, a context longer
- * than the table, or rows outside [0, num_tokens) set PA_DEVERR_CONTEXT_LEN
- * and leave that sequence's rows unwritten; block ids outside the pool are skipped and set
+ * bf16.  Runs on the tensor cores (tcgen05, fp32 accumulation): the softmax
+ * weights P enter P.V in the cache dtype -- for bf16 as a hi + lo pair of
+ * bf16 values (relative rounding ~2^-17 per weight), for fp16 as one fp16
+ * value (2^-11).  No workspace, nothing allocated.  A chunk longer than its
+ * context, a context longer than the table, or rows outside
+ * [0, num_tokens) set PA_DEVERR_CONTEXT_LEN and leave that sequence's rows
+ * unwritten; block ids outside the pool are skipped and set
  * PA_DEVERR_BLOCK_ID.  Rows of a sequence whose C_s is 0 are none.
  */
 int pa_paged_prefill_attention(float *out, const void *q, const void *k_cache,
