@@ -103,16 +103,19 @@ void choose_layout(int D, int B, int G, int sms, int regs_per_thread, DecodeLayo
     const size_t budget = per_sm / c - per_cta_reserved - 256;   // 256: static smem
     return (int)((budget - 1024) / set);
   };
-  // the most CTAs per SM the registers allow that still leave every warp two
-  // stages (a warp streams through its own ring; with one stage it cannot
-  // overlap a copy with the math: measured on B200 at block 32, 64 q / 8 kv
-  // heads, 1 CTA x 2 stages beats 2 CTAs x 1 stage by ~1 %); one stage only
-  // when even a single CTA cannot hold two
-  int ctas = 1;
+  // Every warp streams through its own ring, so the tiles in flight per SM,
+  // CTAs x stages (stages at most 2), are what keep HBM busy: take the most,
+  // and on a tie the layout with more stages, whose warps overlap a copy with
+  // the math (measured on B200 at block 32, 64 q / 8 kv heads: 1 CTA x 2
+  // stages beats 2 CTAs x 1 stage by ~1 %).
+  int ctas = 1, best = 0, best_st = 0;
   for (int c = reg_ctas; c >= 1; --c) {
-    if (stages_for(c) >= 2) {
+    const int st = std::min(stages_for(c), 2);
+    if (st < 1) continue;
+    if (c * st > best || (c * st == best && st > best_st)) {
+      best = c * st;
+      best_st = st;
       ctas = c;
-      break;
     }
   }
   if (want_ctas > 0) ctas = std::min(want_ctas, kMaxCtasPerSm);
