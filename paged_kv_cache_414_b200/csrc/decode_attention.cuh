@@ -93,6 +93,20 @@ struct DecodeParams {
 
 __device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
 
+// L2 policy for data written now and read back by the next kernel: its lines
+// are the last to be evicted.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// Store of one float with an L2 cache policy.
+__device__ __forceinline__ void st_global_hint(float *dst, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(dst), "f"(v), "l"(policy)
+               : "memory");
+}
+
 // Number of blocks of sequence s, with the length clamped into the table.
 template <int B>
 __device__ __forceinline__ int seq_blocks(const DecodeParams &p, int s, bool report) {
@@ -324,6 +338,8 @@ struct MmaPath {
     } else {
       float *po = p.part_o + (int64_t)slot * G * D;
       float *pm = p.part_ml + (int64_t)slot * G * 2;
+      // kept in L2 for the merge kernel that reads it next
+      const uint64_t pol = l2_policy_evict_last();
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -332,12 +348,12 @@ struct MmaPath {
           if (head < G) {
 #pragma unroll
             for (int a = 0; a < KT; ++a) {
-              po[head * D + a * 16 + g] = o[a][n][c];
-              po[head * D + a * 16 + g + 8] = o[a][n][2 + c];
+              st_global_hint(po + head * D + a * 16 + g, o[a][n][c], pol);
+              st_global_hint(po + head * D + a * 16 + g + 8, o[a][n][2 + c], pol);
             }
             if (g == 0) {
-              pm[head * 2 + 0] = m[n][c];
-              pm[head * 2 + 1] = lt[n][c];
+              st_global_hint(pm + head * 2 + 0, m[n][c], pol);
+              st_global_hint(pm + head * 2 + 1, lt[n][c], pol);
             }
           }
         }
@@ -480,12 +496,14 @@ struct ScalarPath {
         *reinterpret_cast<float2 *>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
       }
     } else {
+      // kept in L2 for the merge kernel that reads it next
       float *po = p.part_o + (int64_t)slot * D + lane * DPL;
+      const uint64_t pol = l2_policy_evict_last();
 #pragma unroll
-      for (int k = 0; k < DPL; ++k) po[k] = acc[k];
+      for (int k = 0; k < DPL; ++k) st_global_hint(po + k, acc[k], pol);
       if (lane == 0) {
-        p.part_ml[(int64_t)slot * 2 + 0] = m;
-        p.part_ml[(int64_t)slot * 2 + 1] = lt;
+        st_global_hint(p.part_ml + (int64_t)slot * 2 + 0, m, pol);
+        st_global_hint(p.part_ml + (int64_t)slot * 2 + 1, lt, pol);
       }
     }
   }
@@ -809,8 +827,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   nxt = follow(cur, ntiles - cur.n);
 
   const uint8_t *qbase = p.q;
-  // K/V tiles are read once per call: evict them from L2 first, so the
-  // partials this call writes for the split merge are still there for it.
+  // K/V tiles are read once per call: evict them from L2 first, and the
+  // partials this call writes for the split merge (evict-last) last.
   const uint64_t stream_policy = l2_policy_evict_first();
   auto issue = [&](int stage) {
     if (cur_k == cur.n) {
