@@ -45,12 +45,16 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Grid (chunks, pairs): every block copies `per_block` vectors of one pair's
-// block in both pools.
+// Grid (chunks, pairs): block (x, pair) copies vectors [x * kCopyPerCta,
+// (x + 1) * kCopyPerCta) of the pair's block, in both pools.  Each thread
+// loads all its vectors before it stores any: the caller guarantees that no
+// destination block is also a source, so the loads never see this kernel's
+// stores, and a thread keeps 2 * kCopyUnroll 16-byte loads in flight.
+constexpr int kCopyUnroll = 4;
+constexpr int kCopyPerCta = 256 * kCopyUnroll;
 __global__ void __launch_bounds__(256)
-    copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
-                       const int64_t *__restrict__ block_mapping, long long vec_per_block,
-                       int per_block, int num_blocks) {
+    copy_blocks_kernel(uint4 *k_cache, uint4 *v_cache, const int64_t *__restrict__ block_mapping,
+                       long long vec_per_block, int num_blocks) {
   allow_dependent_launch();
   const long long pair = blockIdx.y;
   const int64_t src = __ldg(block_mapping + 2 * pair);
@@ -59,16 +63,27 @@ __global__ void __launch_bounds__(256)
     if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(PA_DEVERR_COPY_PAIR);
     return;
   }
-  const long long beg = (long long)blockIdx.x * per_block;
-  long long end = beg + per_block;
-  if (end > vec_per_block) end = vec_per_block;
+  const long long beg = (long long)blockIdx.x * kCopyPerCta + threadIdx.x;
   const uint4 *ks = k_cache + src * vec_per_block;
   const uint4 *vs = v_cache + src * vec_per_block;
   uint4 *kd = k_cache + dst * vec_per_block;
   uint4 *vd = v_cache + dst * vec_per_block;
-  for (long long i = beg + threadIdx.x; i < end; i += blockDim.x) {
-    kd[i] = ks[i];
-    vd[i] = vs[i];
+  uint4 kr[kCopyUnroll], vr[kCopyUnroll];
+#pragma unroll
+  for (int u = 0; u < kCopyUnroll; ++u) {
+    const long long i = beg + u * 256;
+    if (i < vec_per_block) {
+      kr[u] = ks[i];
+      vr[u] = vs[i];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kCopyUnroll; ++u) {
+    const long long i = beg + u * 256;
+    if (i < vec_per_block) {
+      kd[i] = kr[u];
+      vd[i] = vr[u];
+    }
   }
 }
 

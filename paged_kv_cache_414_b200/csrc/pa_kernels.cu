@@ -534,12 +534,11 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8))
     return PA_ERR_ARG;
   const long long vec_per_block = (long long)num_kv_heads * block_size * head_dim * 2 / 16;
-  const int per_block = 2048;
-  const unsigned chunks = (unsigned)((vec_per_block + per_block - 1) / per_block);
+  const unsigned chunks = (unsigned)((vec_per_block + pa::kCopyPerCta - 1) / pa::kCopyPerCta);
   dim3 grid(chunks, (unsigned)num_pairs);
   pa::copy_blocks_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
       static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_mapping, vec_per_block,
-      per_block, num_blocks);
+      num_blocks);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
