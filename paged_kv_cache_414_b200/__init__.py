@@ -1,4 +1,4 @@
-"""Python binding of libpa.so, the B200 paged-KV-cache decode library.
+"""Python binding of libpa.so, the B200 paged-KV-cache attention library.
 
 Argument marshalling only: every function here checks the torch tensors it is
 given, passes their device pointers, sizes and the current CUDA stream to the
@@ -7,9 +7,10 @@ the computation runs in Python, and there is no fallback: if libpa.so is
 missing or a call fails, an exception is raised.
 
 Names follow the C ABI: ``pa_reshape_and_cache``, ``pa_paged_decode_attention``
-(with ``pa_paged_decode_workspace_bytes``), ``pa_copy_blocks``,
-``pa_device_error``, and the host block manager ``BlockManager`` over the
-``pa_bm_*`` calls.
+(with ``pa_paged_decode_workspace_bytes``, and ``pa_paged_decode_attention_no_alloc``),
+the fused ``pa_decode_step``, ``pa_paged_prefill_attention`` (chunked prefill),
+``pa_copy_blocks``, ``pa_device_error``, ``pa_decode_tuning``, and the host block
+manager ``BlockManager`` over the ``pa_bm_*`` calls (prefix caching included).
 """
 from __future__ import annotations
 
