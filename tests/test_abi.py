@@ -65,6 +65,8 @@ def test_host_argument_checks(pa):
     assert L.pa_copy_blocks(nul, nul, nul, 0, 8, 128, 16, 10, 1, nul) == 0
     assert L.pa_copy_blocks(nul, nul, nul, 3, 8, 128, 16, 10, 1, nul) == -1
     assert L.pa_copy_blocks(nul, nul, nul, 3, 8, 100, 16, 10, 1, nul) == -2
+    assert L.pa_copy_blocks(nul, nul, nul, 70000, 8, 128, 16, 10, 1, nul) == -2   # > 65535 pairs
+    assert L.pa_copy_blocks(nul, nul, nul, 3, 8, 128, 16, 10, 2, nul) == -1      # fp32 pool
     assert L.pa_decode_tuning(-1, 0, 0) == -1
     assert L.pa_decode_tuning(0, 0, 0) == 0
 
