@@ -54,7 +54,9 @@ WORKLOADS = {
 }
 PREFILL_METRIC = "chunked prefill attention achieved TFLOP/s (% of measured bf16 tensor peak)"
 METRIC = "paged decode attention achieved HBM GB/s (% of B200 peak); decode tokens/s"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_attention_gqa8b.md")
+# committed ncu summaries of the decode kernel, per workload
+PROFILE_SUMMARIES = {w: os.path.join(ROOT, "profiles", f"decode_attention_{w}.md")
+                     for w in ("gqa8b", "13b")}
 KERNEL_SOURCES = ["paged_kv_cache_414_b200/csrc/decode_attention.cuh",
                   "paged_kv_cache_414_b200/csrc/pa_device.cuh"]
 
@@ -88,13 +90,14 @@ def kernel_source_sha(sources=None) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(bytes_per_launch: float):
-    """DRAM bytes (read + write) per launch from the committed ncu summary,
-    scaled from the profiled launch to this run's launches by algorithmic
-    bytes; None unless the summary was taken on the current kernel source."""
+def profiled_traffic(bytes_per_launch: float, workload: str = "gqa8b"):
+    """DRAM bytes (read + write) per launch from the workload's committed ncu
+    summary, scaled from the profiled launch to this run's launches by
+    algorithmic bytes; None without a summary for the workload or unless it
+    was taken on the current kernel source."""
     try:
-        text = open(PROFILE_SUMMARY).read()
-    except OSError:
+        text = open(PROFILE_SUMMARIES[workload]).read()
+    except (KeyError, OSError):
         return None
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     m_tr = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
@@ -448,9 +451,10 @@ def run_b200(args, rank, world, local_rank):
     bytes_launch = float(np.mean(bytes_steps))
     achieved = bytes_launch / (attn_avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
-    # the committed ncu summary is of the gqa8b launch; other workloads run
-    # other kernel instances or (shared prefixes) other DRAM/L2 splits
-    traffic = profiled_traffic(bytes_launch) if args.workload == "gqa8b" else None
+    # from the committed ncu summary of this workload's launch, if there is
+    # one (the others run other kernel instances or, with shared prefixes,
+    # other DRAM/L2 splits)
+    traffic = profiled_traffic(bytes_launch, args.workload)
 
     e2e = None
     if not args.no_e2e:
