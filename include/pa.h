@@ -1,11 +1,13 @@
 /*
- * pa.h -- C ABI of the B200 paged-KV-cache decode library (libpa.so).
+ * pa.h -- C ABI of the B200 paged-KV-cache attention library (libpa.so).
  *
  * The library implements the data-parallel hot path of PagedAttention decode:
  * the KV cache is stored in fixed-size blocks scattered over a physical pool,
  * each sequence owns a block table mapping its logical blocks to physical
  * ones, and attention for the newly generated token reads K/V through that
- * table.  Sources (cited by page title and section):
+ * table; around it, the cache write, copy-on-write block copies, a host block
+ * manager (with prefix caching across requests) and chunked-prefill attention
+ * over the same pool.  Sources (cited by page title and section):
  *
  *   [P1] "Why OS Virtual Memory Paging Saved LLM Inference: The vLLM
  *        Breakthrough" -- section 2 "The PagedAttention Architecture" (KV
@@ -19,8 +21,9 @@
  *
  * Conventions for every call below
  *   - Device pointers are owned by the caller (e.g. torch tensors); the
- *     library never allocates, frees or keeps device memory.  Host pointers
- *     are read or written only during the call.
+ *     library never allocates, frees or keeps device memory (the one fixed
+ *     array of pa_paged_decode_attention_no_alloc is part of the loaded
+ *     module).  Host pointers are read or written only during the call.
  *   - Tensors are dense, row-major ("C-contiguous") in the layouts given.
  *   - Pool layout: k_cache / v_cache are [num_blocks, num_kv_heads,
  *     block_size, head_dim] elements of `dtype`; token t of a sequence lives
