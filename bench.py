@@ -9,6 +9,7 @@ of every sequence through the block tables.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa8b]
     python bench.py --impl reference ...     # the CPU oracle, timed on host cores
     python bench.py --workload prefill       # chunked prefill (tensor cores), TFLOP/s
+    python bench.py --report kv              # paged vs contiguous KV memory (no GPU needed)
 
 Prints one JSON line (rank 0).  `value` is the decode attention's algorithmic
 HBM bytes (every K/V element of every cached token read once, plus the block
@@ -57,8 +58,11 @@ METRIC = "paged decode attention achieved HBM GB/s (% of B200 peak); decode toke
 # committed ncu summaries of the decode kernel, per workload
 PROFILE_SUMMARIES = {w: os.path.join(ROOT, "profiles", f"decode_attention_{w}.md")
                      for w in ("gqa8b", "13b")}
+# sources that decide a kernel's DRAM traffic: the kernel itself and the host
+# code that picks its launch shape (grid, CTAs per SM, stages, scratch layout)
 KERNEL_SOURCES = ["paged_kv_cache_414_b200/csrc/decode_attention.cuh",
-                  "paged_kv_cache_414_b200/csrc/pa_device.cuh"]
+                  "paged_kv_cache_414_b200/csrc/pa_device.cuh",
+                  "paged_kv_cache_414_b200/csrc/pa_kernels.cu"]
 
 
 def parse():
@@ -71,6 +75,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--report", choices=["kv"], default=None,
+                    help="print the KV memory report (paged vs contiguous) instead of timing")
     return ap.parse_args()
 
 
@@ -79,7 +85,8 @@ def parse():
 PREFILL_PROFILE = os.path.join(ROOT, "profiles", "prefill_attention_16x512.md")
 PREFILL_SOURCES = ["paged_kv_cache_414_b200/csrc/prefill_attention.cuh",
                    "paged_kv_cache_414_b200/csrc/umma.cuh",
-                   "paged_kv_cache_414_b200/csrc/pa_device.cuh"]
+                   "paged_kv_cache_414_b200/csrc/pa_device.cuh",
+                   "paged_kv_cache_414_b200/csrc/pa_kernels.cu"]
 
 
 def kernel_source_sha(sources=None) -> str:
@@ -218,6 +225,28 @@ def rank_reduce(x: float, op: str, world: int, device=None) -> float:
     return float(t.item())
 
 
+def decode_bytes(context_lens, num_kv_heads: int, head_dim: int, block_size: int,
+                 elem_bytes: int = 2) -> int:
+    """Algorithmic HBM bytes of one decode-attention call: every cached K and V
+    element of every sequence read once, plus the block-table entries used."""
+    total = 0
+    for L in np.asarray(context_lens).tolist():
+        L = int(L)
+        total += 2 * L * num_kv_heads * head_dim * elem_bytes + 4 * math.ceil(L / block_size)
+    return total
+
+
+def prefill_flops(context_lens, chunk_lens, num_q_heads: int, head_dim: int) -> int:
+    """Algorithmic FLOPs of one chunked-prefill attention call: a chunk token
+    at position p costs 2*head_dim*(p+1) for its scores and as much for P.V,
+    per query head; positions run L-C .. L-1, so a sequence contributes
+    4*D*Hq * C*(2L - C + 1)/2."""
+    total = 0
+    for L, C in zip(np.asarray(context_lens).tolist(), np.asarray(chunk_lens).tolist()):
+        total += 4 * head_dim * num_q_heads * (int(C) * (2 * int(L) - int(C) + 1) // 2)
+    return total
+
+
 def rank_seed(name: str, rank: int) -> int:
     """Each rank draws its own independent batch (weak scaling)."""
     return W.SEEDS[name] + 1000 * rank
@@ -283,7 +312,6 @@ class Workload:
     def bytes_per_step(self, step: int) -> int:
         """Algorithmic (logical) bytes: every cached token of every sequence;
         for shared prompt blocks that is once per branch reading them."""
-        from paged_kv_cache_414_b200 import decode_bytes
         return decode_bytes(self.lens0 + step, self.shape.num_kv_heads, self.shape.head_dim,
                             self.shape.block_size, self.elem)
 
@@ -326,6 +354,33 @@ class Workload:
                 for s in range(self.S):
                     bm.append_slot(s)
         return bm, [bm.append_slot(s)[0] for s in range(self.S)]
+
+
+def decode_config(wl, name: str, world: int, K: int, Wm: int) -> dict:
+    """The `config` of a decode line; both arms print the same one."""
+    sh = wl.shape
+    timed = (lambda k: k) if wl.cyclic else (lambda k: Wm + k)  # noqa: E731
+    b = wl.batch
+    pool_bytes = 2 * b.k_cache.numel() * b.k_cache.element_size()
+    flush = pool_bytes < 2 * 126 * 2 ** 20
+    bytes_launch = float(np.mean([wl.bytes_per_step(timed(k)) for k in range(K)]))
+    return {
+        "workload": f"{name}: {WORKLOADS[name]}",
+        "num_seqs_per_gpu": wl.S,
+        "num_q_heads": sh.num_q_heads,
+        "num_kv_heads": sh.num_kv_heads,
+        "head_dim": sh.head_dim,
+        "block_size": sh.block_size,
+        "mean_context_len": float(np.mean(wl.lens0)) + float(np.mean([timed(k) for k in range(K)])),
+        "bytes_per_step": bytes_launch,
+        "parallelism": f"dp{world} (independent batches, no collective on the data path)",
+        "l2": ("K/V pool %.0f MB, under twice L2: L2 flushed (256 MB memset) before "
+               "every timed step, outside the per-step CUDA-event spans" % (pool_bytes / 1e6)
+               if flush else "inputs larger than L2: %.2f GB of KV read per step, no flush"
+               % (bytes_launch / 1e9)),
+        "step": "host block manager (prepared ahead) -> copy_blocks if any -> pa_decode_step "
+                "(cache write of the new token + paged decode attention) -> split merge",
+    }
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -478,22 +533,7 @@ def run_b200(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": sh.dtype,
             "data": "synthetic",
-            "config": {
-                "workload": f"{args.workload}: {WORKLOADS[args.workload]}",
-                "num_seqs_per_gpu": S,
-                "num_q_heads": sh.num_q_heads,
-                "num_kv_heads": sh.num_kv_heads,
-                "head_dim": sh.head_dim,
-                "block_size": B,
-                "mean_context_len": float(np.mean(wl.lens0)) + float(np.mean(
-                    [timed_idx(k) for k in range(K)])),
-                "parallelism": f"dp{world} (independent batches, no collective on the data path)",
-                "l2": ("K/V pool %.0f MB, under twice L2: L2 flushed (256 MB memset) before "
-                       "every timed step, outside the per-step CUDA-event spans" % (pool_bytes / 1e6)
-                       if flush else "inputs larger than L2: %.2f GB of KV read per step, no flush"
-                       % (bytes_launch / 1e9)),
-                "step": "host block manager (prepared ahead) -> copy_blocks if any -> pa_decode_step (cache write of the new token + paged decode attention) -> split merge",
-            },
+            "config": decode_config(wl, args.workload, world, K, Wm),
             "pct_of_measured_hbm_peak": round(100.0 * value / peak / world, 2),
             "pct_of_nominal_8tbs": round(100.0 * value / 8000.0 / world, 2),
             "decode_tokens_per_s": round(tokens_per_s, 1),
@@ -661,8 +701,31 @@ class PrefillBench:
         bm.close()
         assert np.array_equal(tables, b.block_tables) and np.array_equal(ctx, b.context_lens)
         self.slots = np.concatenate(slots).astype(np.int64)
-        self.flops = pa.prefill_flops(lens, chunks, self.shape.num_q_heads, self.shape.head_dim)
+        self.flops = prefill_flops(lens, chunks, self.shape.num_q_heads, self.shape.head_dim)
         self.max_query_len = int(chunks.max())
+
+
+def prefill_config(pb, world: int) -> dict:
+    """The `config` of a prefill line; both arms print the same one."""
+    b, sh = pb.batch, pb.shape
+    return {
+        "workload": f"prefill: {WORKLOADS['prefill']}",
+        "num_seqs_per_gpu": b.num_seqs,
+        "num_tokens_per_step": b.num_tokens,
+        "num_q_heads": sh.num_q_heads,
+        "num_kv_heads": sh.num_kv_heads,
+        "head_dim": sh.head_dim,
+        "block_size": sh.block_size,
+        "mean_context_len": float(np.mean(b.context_lens)),
+        "flops_per_step": pb.flops,
+        "parallelism": f"dp{world} (independent batches, no collective on the data path)",
+        "l2": "inputs larger than L2 (%.0f MB of K/V pool, %.0f MB of q, %.0f MB of "
+              "output per step), no flush" % (
+                  2 * b.k_cache.numel() * 2 / 1e6, b.q.numel() * 2 / 1e6,
+                  b.num_tokens * sh.num_q_heads * sh.head_dim * 4 / 1e6),
+        "step": "reshape_and_cache of the chunk (slots prepared ahead by the host block "
+                "manager) -> pa_paged_prefill_attention",
+    }
 
 
 def run_prefill_b200(args, rank, world, local_rank):
@@ -752,23 +815,7 @@ def run_prefill_b200(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": sh.dtype,
             "data": "synthetic",
-            "config": {
-                "workload": f"prefill: {WORKLOADS['prefill']}",
-                "num_seqs_per_gpu": b.num_seqs,
-                "num_tokens_per_step": T,
-                "num_q_heads": sh.num_q_heads,
-                "num_kv_heads": sh.num_kv_heads,
-                "head_dim": sh.head_dim,
-                "block_size": sh.block_size,
-                "mean_context_len": float(np.mean(b.context_lens)),
-                "parallelism": f"dp{world} (independent batches, no collective on the data path)",
-                "l2": "inputs larger than L2 (%.0f MB of K/V pool, %.0f MB of q, %.0f MB of "
-                      "output per step), no flush" % (
-                          2 * b.k_cache.numel() * 2 / 1e6, b.q.numel() * 2 / 1e6,
-                          out.numel() * 4 / 1e6),
-                "step": "reshape_and_cache of the chunk (slots prepared ahead by the host block "
-                        "manager) -> pa_paged_prefill_attention",
-            },
+            "config": prefill_config(pb, world),
             "pct_of_measured_bf16_peak": round(100.0 * value / peak / world, 2),
             "roofline": {
                 "bound": "tensor",
@@ -893,7 +940,6 @@ def prefill_oracle_sample(pb, seqs, kb, vb):
                                b.query_start, b.scale, sh.num_kv_heads, sh.block_size, sh.dtype,
                                seqs=seqs)
     dt = time.perf_counter() - t0
-    from paged_kv_cache_414_b200 import prefill_flops
     return dt, prefill_flops(b.context_lens[seqs], b.chunk_lens[seqs], sh.num_q_heads,
                              sh.head_dim)
 
@@ -943,16 +989,12 @@ def run_prefill_reference(args, rank, world):
             times.append(dt)
             flops.append(f)
     value = sum(flops) / sum(times) / 1e12
-    sh = pb.shape
     line = {
         "impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6),
         "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": Wm,
         "ms_per_step": round(1e3 * sum(times) / K, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"prefill: {WORKLOADS['prefill']}",
-                   "num_seqs_per_gpu": pb.batch.num_seqs, "num_q_heads": sh.num_q_heads,
-                   "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
-                   "block_size": sh.block_size, "parallelism": "host cores"},
+        "config": prefill_config(pb, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores_used(),
                          "kind": "oracle",
                          "sample": "one sequence of the prefill batch per step (fp64 attention "
@@ -961,6 +1003,97 @@ def run_prefill_reference(args, rank, world):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- KV memory report
+
+# The pages' figures the report is set beside (context, not targets).
+PAGES_KV_FIGURES = {
+    "prior_systems_useful_kv_fraction": [0.20, 0.38],
+    "prior_systems_useful_source": "vLLM & PagedAttention: OS Ideas for LLM Serving, section 01 "
+                                   "'The Problem' (the 2023 paper's measurement)",
+    "prior_systems_memory_wasted_fraction": [0.60, 0.80],
+    "prior_systems_wasted_source": "Why OS Virtual Memory Paging Saved LLM Inference, "
+                                   "introduction; vLLM & PagedAttention, introduction",
+    "paged_waste_fraction_below": 0.04,
+    "paged_waste_source": "Why OS Virtual Memory Paging Saved LLM Inference, section 3",
+    "example": {"reserved_tokens": 2048, "used_tokens": 150, "idle_slots": 1898,
+                "source": "Why OS Virtual Memory Paging Saved LLM Inference, section 1"},
+}
+
+
+def kv_accounting(stats: dict, reserve: int) -> dict:
+    """KV memory of a block manager's live sequences (its pa_bm_stats) against
+    a contiguous reservation of `reserve` tokens per sequence, the allocation
+    paged blocks replace: slots allocated, the fraction holding tokens, idle
+    slots.  A block shared by several sequences is one allocation whose
+    filled slots count once; a contiguous reservation shares nothing, so
+    every sequence's tokens are stored (and useful) in its own buffer."""
+    B = stats["block_size"]
+    paged = stats["used_blocks"] * B
+    filled = stats["filled_slots"]
+    tokens = stats["logical_tokens"]
+    contiguous = stats["num_seqs"] * reserve
+    return {
+        "sequences": stats["num_seqs"],
+        "logical_tokens": tokens,
+        "paged_slots": paged,
+        "paged_filled_slots": filled,
+        "paged_idle_slots": paged - filled,
+        "paged_useful_fraction": filled / paged if paged else 1.0,
+        "paged_waste_fraction": (paged - filled) / paged if paged else 0.0,
+        "shared_blocks": stats["shared_blocks"],
+        "sharing_ratio": tokens / filled if filled else 1.0,
+        "contiguous_reserve_tokens": reserve,
+        "contiguous_slots": contiguous,
+        "contiguous_idle_slots": contiguous - tokens,
+        "contiguous_useful_fraction": tokens / contiguous if contiguous else 1.0,
+        "paged_slots_per_contiguous_slot": paged / contiguous if contiguous else 0.0,
+    }
+
+
+def kv_report(pa) -> dict:
+    """Paged versus contiguous KV memory on the workloads' length mixes, from
+    the native block manager's own accounting (pa_bm_stats)."""
+    out = {"report": "kv_utilisation", "source": "pa_bm_stats of the native block manager",
+           "pages": PAGES_KV_FIGURES, "workloads": {}}
+    # the pages' worked example through the manager: one 150-token request
+    bm = pa.BlockManager(16, 16)
+    bm.allocate(0, 150)
+    out["workloads"]["example_150_tokens"] = dict(
+        kv_accounting(bm.stats(), 2048), reserve_reason="the pages' 2,048-token reservation")
+    bm.close()
+    reserves = {"13b": (2048, "the workload's longest context"),
+                "gqa8b": (4096, "the workload's longest context"),
+                "long": (32768, "the workload's longest context")}
+    for name, (reserve, why) in reserves.items():
+        sh = W.SHAPES[name]
+        lens = {"13b": W.lens_13b, "gqa8b": W.lens_gqa8b,
+                "long": W.lens_long}[name](np.random.default_rng(W.SEEDS[name]))
+        nblk = int(sum(-(-int(L) // sh.block_size) for L in lens))
+        bm = pa.BlockManager(nblk, sh.block_size)
+        for s, L in enumerate(lens):
+            bm.allocate(s, int(L))
+        out["workloads"][name] = dict(kv_accounting(bm.stats(), reserve), reserve_reason=why)
+        bm.close()
+    # parallel sampling: prompts shared by their 8 branches, then 64 decode
+    # steps with copy-on-write of the shared partial last blocks
+    cw = W.cow_workload()
+    B = cw.shape.block_size
+    bm = pa.BlockManager(cw.num_blocks, B, cw.free_order)
+    for p_, P in enumerate(cw.prompt_lens):
+        bm.allocate(cw.seq_id(p_, 0), int(P))
+        for br in range(1, cw.branches):
+            bm.fork(cw.seq_id(p_, 0), cw.seq_id(p_, br))
+    why = "the pages' 2,048-token reservation per branch (contexts reach 576 tokens)"
+    out["workloads"]["cow_after_fork"] = dict(kv_accounting(bm.stats(), 2048), reserve_reason=why)
+    seqs = np.arange(cw.num_seqs)
+    for _ in range(cw.steps):
+        bm.append_slots(seqs)
+    out["workloads"]["cow_after_64_steps"] = dict(kv_accounting(bm.stats(), 2048),
+                                                  reserve_reason=why)
+    bm.close()
+    return out
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
@@ -992,7 +1125,6 @@ def oracle_step_sample(wl, step: int, seqs):
         lens[i] = bm.seq_len(s)
     OA.paged_decode_attention(qb, kb, vb, tabs, lens, wl.scale, sh.num_kv_heads, B, sh.dtype)
     dt = time.perf_counter() - t0
-    from paged_kv_cache_414_b200 import decode_bytes
     return dt, decode_bytes(lens, sh.num_kv_heads, sh.head_dim, B, 2)
 
 
@@ -1037,7 +1169,6 @@ def run_reference(args, rank, world):
             times.append(dt)
             nbytes.append(nb)
     value = sum(nbytes) / sum(times) / 1e9
-    sh = wl.shape
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -1052,10 +1183,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}",
-                   "num_seqs_per_gpu": wl.S, "num_q_heads": sh.num_q_heads,
-                   "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
-                   "block_size": sh.block_size, "parallelism": "host cores"},
+        "config": decode_config(wl, args.workload, world, K, Wm),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_cores_used(),
                          "kind": "oracle",
                          "sample": f"{nseq} of {wl.S} sequences per step (oracle cache write + "
@@ -1071,6 +1199,13 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.report == "kv":
+        if rank == 0:
+            from paged_kv_cache_414_b200 import build as pbuild
+            pbuild.build()
+            import paged_kv_cache_414_b200 as pa
+            print(json.dumps(kv_report(pa)), flush=True)
+        return
     if args.impl == "reference":
         if args.workload == "prefill":
             run_prefill_reference(args, rank, world)

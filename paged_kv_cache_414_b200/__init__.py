@@ -9,13 +9,13 @@ missing or a call fails, an exception is raised.
 Names follow the C ABI: ``pa_reshape_and_cache``, ``pa_paged_decode_attention``
 (with ``pa_paged_decode_workspace_bytes``, and ``pa_paged_decode_attention_no_alloc``),
 the fused ``pa_decode_step``, ``pa_paged_prefill_attention`` (chunked prefill),
-``pa_copy_blocks``, ``pa_device_error``, ``pa_decode_tuning``, and the host block
-manager ``BlockManager`` over the ``pa_bm_*`` calls (prefix caching included).
+``pa_copy_blocks``, ``pa_device_error``, ``pa_decode_tuning``, ``pa_set_wait_limit``,
+and the host block manager ``BlockManager`` over the ``pa_bm_*`` calls (prefix
+caching included).
 """
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 import numpy as np
@@ -80,6 +80,7 @@ def _declare(L):
         "pa_decode_step": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                  i32, i32, i32, i32, vp, sz, vp]),
         "pa_decode_tuning": (i32, [i32, i32, i32]),
+        "pa_set_wait_limit": (i32, [c.c_longlong]),
         "pa_paged_prefill_attention": (i32, [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32,
                                              i32, i32, i32, i32, i32, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
@@ -304,6 +305,11 @@ def pa_decode_tuning(nstage=0, ctas_per_sm=0, min_tiles_per_warp=0):
     _check(lib().pa_decode_tuning(nstage, ctas_per_sm, min_tiles_per_warp), "pa_decode_tuning")
 
 
+def pa_set_wait_limit(ns: int = 0):
+    """Limit (ns) of every bounded wait in kernels launched afterwards; 0 = the default 2 s."""
+    _check(lib().pa_set_wait_limit(int(ns)), "pa_set_wait_limit")
+
+
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
     """k_cache[dst] = k_cache[src] (and V) for every (src, dst) row of block_mapping."""
     torch = _torch()
@@ -468,52 +474,8 @@ class BlockManager:
         return lib().pa_bm_num_seqs(self._h)
 
     def stats(self) -> dict:
-        """pa_bm_stats: blocks used / shared / free, tokens, filled slots, plus
-        the derived idle slots and waste fraction."""
+        """pa_bm_stats as a dict: blocks (total, free, used, shared), live
+        sequences, logical tokens, filled slots, block size."""
         st = BmStats()
         _check(lib().pa_bm_stats(self._h, ctypes.byref(st)), "pa_bm_stats")
-        d = {name: int(getattr(st, name)) for name, _ in BmStats._fields_}
-        slots = d["used_blocks"] * d["block_size"]
-        d["idle_slots"] = slots - d["filled_slots"]
-        d["waste_fraction"] = d["idle_slots"] / slots if slots else 0.0
-        return d
-
-
-def utilisation_report(bm: "BlockManager", reserve: int) -> dict:
-    """Paged KV memory of the manager's live sequences against a contiguous
-    reservation of `reserve` tokens per sequence (the allocation PagedAttention
-    replaces): slots allocated, useful fraction, idle slots, for both."""
-    st = bm.stats()
-    contiguous = st["num_seqs"] * reserve
-    paged = st["used_blocks"] * st["block_size"]
-    return {
-        "paged_slots": paged,
-        "paged_useful_fraction": st["filled_slots"] / paged if paged else 1.0,
-        "paged_idle_slots": st["idle_slots"],
-        "contiguous_slots": contiguous,
-        "contiguous_useful_fraction": st["logical_tokens"] / contiguous if contiguous else 1.0,
-        "contiguous_idle_slots": contiguous - st["logical_tokens"],
-        "sharing_ratio": st["logical_tokens"] / st["filled_slots"] if st["filled_slots"] else 1.0,
-    }
-
-
-def decode_bytes(context_lens, num_kv_heads: int, head_dim: int, block_size: int,
-                 elem_bytes: int = 2) -> int:
-    """Algorithmic HBM bytes of one decode-attention call: every cached K and V
-    element of every sequence read once plus the block-table entries used."""
-    total = 0
-    for L in np.asarray(context_lens).tolist():
-        L = int(L)
-        total += 2 * L * num_kv_heads * head_dim * elem_bytes + 4 * math.ceil(L / block_size)
-    return total
-
-
-def prefill_flops(context_lens, chunk_lens, num_q_heads: int, head_dim: int) -> int:
-    """Algorithmic FLOPs of one chunked-prefill attention call: a chunk token
-    at position p costs 2*head_dim*(p+1) for its scores and as much for P.V,
-    per query head; positions run L-C .. L-1, so a sequence contributes
-    4*D*Hq * C*(2L - C + 1)/2."""
-    total = 0
-    for L, C in zip(np.asarray(context_lens).tolist(), np.asarray(chunk_lens).tolist()):
-        total += 4 * head_dim * num_q_heads * (int(C) * (2 * int(L) - int(C) + 1) // 2)
-    return total
+        return {name: int(getattr(st, name)) for name, _ in BmStats._fields_}
