@@ -101,10 +101,13 @@ int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void
                          pa_stream_t stream);
 
 /*
- * Bytes of device workspace pa_paged_decode_attention needs on the current
- * device for these sizes (0 on error).  The workspace holds the per-warp
- * split-context partial results and their descriptors; its contents need no
- * initialisation and are dead after the call.
+ * Bytes of device workspace that cover every pa_paged_decode_attention or
+ * pa_decode_step launch on the current device for these sizes, whatever
+ * pa_decode_tuning selects (0 on error): an upper bound, sized for the
+ * largest grid (4 CTAs per SM); the default launch needs less.  The
+ * workspace holds the per-warp split-context partial results and their
+ * descriptors; its contents need no initialisation and are dead after the
+ * call.
  */
 size_t pa_paged_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
                                        int head_dim, int block_size, int max_context_len);
@@ -122,7 +125,9 @@ size_t pa_paged_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv
  * accumulated in fp32.  L counts every cached token of the sequence, the one
  * written this step included; L == 0 gives a zero row.  Long sequences are
  * split across warps (split context) and the partial softmax states are
- * merged by a second kernel launched on the same stream.
+ * merged by a second kernel launched on the same stream.  If a bounded wait
+ * of the call runs out (PA_DEVERR_TIMEOUT, see pa_set_wait_limit), its output
+ * rows are undefined.
  *
  *   out           fp32 [num_seqs, num_q_heads, head_dim] (device, written)
  *   q             dtype [num_seqs, num_q_heads, head_dim] (device)
@@ -185,12 +190,24 @@ int pa_decode_step(float *out, const void *q, const void *k_new, const void *v_n
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  Every call on a device shares the one array, which keeps the
- * last call's contents (nothing in it needs clearing between calls): calls
- * that may overlap on the GPU -- on different streams, or from different
- * threads -- race and must be serialised by the caller.  Returns
- * PA_ERR_WORKSPACE when the launch would need more than
- * PA_NO_ALLOC_SCRATCH_BYTES (pa_paged_decode_workspace_bytes tells the need);
- * otherwise as pa_paged_decode_attention.
+ * last call's contents: every partial result the call reads back is written
+ * by the same call first, so nothing needs clearing between calls (after a
+ * call whose wait ran out, PA_DEVERR_TIMEOUT, the output is undefined
+ * anyway).  Calls that may overlap on the GPU -- on different streams, or
+ * from different threads -- race on the array and must be serialised by the
+ * caller.  Returns PA_ERR_WORKSPACE, launching nothing, when the launch
+ * would need more than PA_NO_ALLOC_SCRATCH_BYTES; otherwise as
+ * pa_paged_decode_attention.
+ *
+ * What fits: the scratch of a launch is about 8 * W * (G * (head_dim + 2) + 8)
+ * bytes for W warps in the grid and G = num_q_heads / num_kv_heads (it does
+ * not depend on the number of sequences or their lengths).  With the default
+ * launch shape on a 148-SM B200 (W = 1184 for G >= 2 at block_size 16 or at
+ * head_dim 64, W = 592 at head_dim 128 with block_size 32, W = 1776 for
+ * G = 1) every supported shape fits except head_dim 128, block_size 16 with
+ * G = 14, 15 or 16.  pa_paged_decode_workspace_bytes is an upper bound over
+ * all tunings, not this launch's need: it exceeds the array from G = 7 at
+ * head_dim 128 although those calls succeed.
  */
 #define PA_NO_ALLOC_SCRATCH_BYTES (16u << 20)
 int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_cache,
@@ -209,6 +226,20 @@ int pa_paged_decode_attention_no_alloc(float *out, const void *q, const void *k_
  * hence the rounding, change.  No counterpart on the pages: a tuning knob.
  */
 int pa_decode_tuning(int nstage, int ctas_per_sm, int min_tiles_per_warp);
+
+/*
+ * Limit, in nanoseconds of wall time, of every bounded wait inside the
+ * kernels launched after this call (decode, decode step, prefill): a wait on
+ * an asynchronous copy or on the tensor cores that lasts longer gives up,
+ * sets PA_DEVERR_TIMEOUT, lets the copies and MMAs already issued complete
+ * (those drains keep their own fixed bounds, so nothing lands after a CTA
+ * has left) and returns; the output rows of that call are then undefined.
+ * ns == 0 restores the default of 2 s, far above any copy's latency; a tiny
+ * limit makes the waits run out on purpose, which is how failure detection
+ * is tested without faulting or hanging the GPU.  Process-wide; returns
+ * PA_ERR_ARG for ns < 0.  No counterpart on the pages.
+ */
+int pa_set_wait_limit(long long ns);
 
 /*
  * Copy-on-write block copies ([P1] section 3: a branch that writes into a
@@ -255,7 +286,7 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
  * head_dim 64 or 128, block_size 16 or 32, group size up to 16, fp16 or
  * bf16.  Runs on the tensor cores (tcgen05, fp32 accumulation): the softmax
  * weights P enter P.V in the cache dtype -- for bf16 as a hi + lo pair of
- * bf16 values (relative rounding ~2^-17 per weight), for fp16 as one fp16
+ * bf16 values (relative error under 2^-14 per weight), for fp16 as one fp16
  * value (2^-11).  No workspace, nothing allocated.  A chunk longer than its
  * context, a context longer than the table, or rows outside
  * [0, num_tokens) set PA_DEVERR_CONTEXT_LEN and leave that sequence's rows

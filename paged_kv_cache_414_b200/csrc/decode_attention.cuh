@@ -50,7 +50,6 @@
 
 namespace pa {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a copy never takes this long
 constexpr uint64_t kDrainLimitNs = 20000000ull;    // 20 ms to drain after a time-out
 constexpr int kMetaWords = 8;                      // per-warp descriptor for the merge
 
@@ -89,6 +88,7 @@ struct DecodeParams {
   int max_blocks, num_blocks;
   int nstage;
   int min_tiles;       // fewest tiles a warp is given
+  uint64_t wait_ns;    // limit of a wait on a copy before giving up (2 s by default)
 };
 
 __device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
@@ -903,10 +903,11 @@ __global__ void __launch_bounds__(NW * 32, NT == 0 ? 3 : 2)
   for (long long i = 0; i < ntiles; ++i) {
     const int stage = (int)(i % nstage);
     const uint32_t parity = (uint32_t)((i / nstage) & 1);
-    if (!mbar_wait_bounded(&bars[stage], parity, kWaitLimitNs)) {
+    if (!mbar_wait_bounded(&bars[stage], parity, p.wait_ns)) {
       if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
-      // drain the copies still in flight, then leave
-      for (long long k = i + 1; k < i + nstage && k < issued; ++k)
+      // drain the copies still in flight -- this tile's and those issued
+      // after it -- so that none lands after the warp has left
+      for (long long k = i; k < issued; ++k)
         mbar_wait_bounded(&bars[k % nstage], (uint32_t)((k / nstage) & 1), kDrainLimitNs);
       return;
     }

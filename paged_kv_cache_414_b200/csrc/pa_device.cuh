@@ -69,15 +69,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait whose suspension lasts at most `hint_ns` (instead of the
+// hardware's own limit), so that a short wait limit can run out while the
+// awaited copy is still in flight.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Limits at or above this keep the plain try_wait (the normal case: 2 s).
+constexpr uint64_t kShortWaitNs = 1000000ull;
+
+// One try_wait within a wait limited to `limit_ns`.
+__device__ __forceinline__ bool mbar_try_wait_within(uint64_t *bar, uint32_t parity,
+                                                     uint64_t limit_ns) {
+  if (limit_ns >= kShortWaitNs) return mbar_try_wait(bar, parity);
+  return mbar_try_wait_hint(bar, parity, (uint32_t)limit_ns);
+}
+
 // Wait for the barrier phase with the given parity to complete, giving up
 // after `limit_ns` of wall time.  Returns false on time-out (the caller sets
 // PA_DEVERR_TIMEOUT and winds down).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }

@@ -55,6 +55,11 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Limit of every bounded wait on an asynchronous copy or MMA in the kernels
+// launched from now on (pa_set_wait_limit).
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;   // 2 s
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+
 // User overrides of the launch heuristics (0 = automatic).
 std::atomic<int> g_tune_nstage{0};
 std::atomic<int> g_tune_ctas{0};
@@ -209,6 +214,7 @@ int launch_decode(const DecodeArgs &a, int dev, int sms) {
   p.num_blocks = a.num_blocks;
   p.nstage = L.nstage;
   p.min_tiles = L.min_tiles;
+  p.wait_ns = g_wait_limit_ns.load();
 
   // Programmatic dependent launch: the grid may be scheduled while the
   // previous kernel on the stream (typically reshape_and_cache) is still
@@ -331,6 +337,7 @@ int launch_prefill(const PrefillArgs &a, int dev) {
   p.num_blocks = a.num_blocks;
   p.tq = tq;
   p.q_tiles = (a.max_query_len + 2 * tq - 1) / (2 * tq);   // a CTA takes two query tiles
+  p.wait_ns = g_wait_limit_ns.load();
   const long long nx = (long long)p.q_tiles * a.num_seqs;
   if (nx >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
   cudaLaunchConfig_t cfg = {};
@@ -625,6 +632,12 @@ int pa_paged_prefill_attention(float *out, const void *q, const void *k_cache,
                 max_query_len, num_blocks, (cudaStream_t)stream};
   if (dtype == PA_BF16) return dispatch_prefill<__nv_bfloat16>(a, dev);
   return dispatch_prefill<__half>(a, dev);
+}
+
+int pa_set_wait_limit(long long ns) {
+  if (ns < 0) return PA_ERR_ARG;
+  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : (unsigned long long)ns);
+  return PA_OK;
 }
 
 int pa_decode_tuning(int nstage, int ctas_per_sm, int min_tiles_per_warp) {

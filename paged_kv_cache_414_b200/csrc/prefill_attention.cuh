@@ -36,8 +36,9 @@
 //               partial sums once at the end.  Online maximum and sum in
 //               fp32; the weights go to tensor memory, where the P.V MMA reads
 //               them as its A operand.  For bf16, P = P_hi + P_lo (both bf16, two
-//               MMAs), so P carries about 2^-17 relative rounding instead of
-//               bf16's 2^-9; for fp16 one fp16 P whose rounded weights are
+//               MMAs, each cut from the fp32 weight by bit operations), so P
+//               carries under 2^-14 relative error instead of bf16's 2^-9;
+//               for fp16 one fp16 P whose rounded weights are
 //               also what the sum adds.  O is rescaled in tensor memory when
 //               the row maximum moves by more than 2^8; the epilogue writes
 //               out = O / l.
@@ -69,13 +70,14 @@ struct PrefillParams {
   int num_seqs, num_tokens, num_q_heads, num_kv_heads, group, max_blocks, num_blocks;
   int q_tiles;                   // CTAs (pairs of query tiles) per sequence in the grid
   int tq;                        // chunk tokens per query tile (128 / group)
+  uint64_t wait_ns;              // limit of a wait before giving up (2 s by default)
 };
 
 constexpr int kPfRows = 128;      // query rows per query tile
 constexpr int kPfKeys = 128;      // keys per K/V tile
 constexpr int kPfThreads = 576;   // producer warp, MMA warp, 2 x 8 softmax warps
 constexpr uint32_t kPfTmemCols = 512;
-constexpr uint64_t kPfWaitLimitNs = 2000000000ull;
+constexpr uint64_t kPfDrainLimitNs = 2000000000ull;   // draining after an abort
 
 template <int D>
 struct PrefillSmem {
@@ -93,13 +95,14 @@ struct PrefillSmem {
 };
 
 // Bounded wait that also gives up when another role has aborted.
-__device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                        uint64_t limit_ns) {
+  if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kPfWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       flag_error(PA_DEVERR_TIMEOUT);
       return false;
@@ -122,13 +125,16 @@ template <>
 struct PfPack<__nv_bfloat16> {
   static constexpr bool kBf16 = true;
   static constexpr bool kSplit = true;     // P = hi + lo
-  // (a, b) -> packed hi pair, packed lo pair (the rounding remainders)
+  // (a, b) -> packed hi pair, packed lo pair.  hi is each weight cut to bf16
+  // (its upper 16 bits), lo the exact remainder cut to bf16 the same way, so
+  // hi + lo is the weight within 2^-14 relative; bit operations and fp32
+  // subtractions only, no conversion instructions.
   __device__ __forceinline__ static void split2(float a, float b, uint32_t *hi, uint32_t *lo) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    float2 f = __bfloat1622float2(h);
-    __nv_bfloat162 r = __floats2bfloat162_rn(a - f.x, b - f.y);
-    *hi = *reinterpret_cast<uint32_t *>(&h);
-    *lo = *reinterpret_cast<uint32_t *>(&r);
+    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    *hi = __byte_perm(ua, ub, 0x7632);
+    const float ra = a - __uint_as_float(ua & 0xffff0000u);
+    const float rb = b - __uint_as_float(ub & 0xffff0000u);
+    *lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
   }
   __device__ __forceinline__ static uint32_t round2(float a, float b, float *sum) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       if (bad && cc == 0 && ckv == 0) flag_error(PA_DEVERR_BLOCK_ID);
       if (j >= NST) {
-        const bool w = lane == 0 ? pf_wait(&empty[st], (j / NST - 1) & 1, abort) : true;
+        const bool w = lane == 0 ? pf_wait(&empty[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
         if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
       const unsigned valid = __ballot_sync(0xffffffffu, id >= 0);
@@ -294,10 +300,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // copies still in flight must land before the CTA exits
     if (lane == 0) {
       for (int j = max(0, issued - NST); j < issued; ++j) {
-        mbar_wait_bounded(&full_k[j % NST], (j / NST) & 1, kPfWaitLimitNs);
-        mbar_wait_bounded(&full_v[j % NST], (j / NST) & 1, kPfWaitLimitNs);
+        mbar_wait_bounded(&full_k[j % NST], (j / NST) & 1, kPfDrainLimitNs);
+        mbar_wait_bounded(&full_v[j % NST], (j / NST) & 1, kPfDrainLimitNs);
       }
-      mbar_wait_bounded(q_full, 0, kPfWaitLimitNs);
+      mbar_wait_bounded(q_full, 0, kPfDrainLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         umma_commit(&o_done[x]);
       };
-      bool ok = pf_wait(q_full, 0, abort) && pf_wait(&full_k[0], 0, abort);
+      bool ok = pf_wait(q_full, 0, abort, p.wait_ns) && pf_wait(&full_k[0], 0, abort, p.wait_ns);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -337,25 +343,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         // tile A: its P.V, then its next S (which overwrites its P, in issue order)
-        if (!pf_wait(&p_full[0], j & 1, abort)) break;
-        if (!pf_wait(&full_v[j % NST], (j / NST) & 1, abort)) break;
+        if (!pf_wait(&p_full[0], j & 1, abort, p.wait_ns)) break;
+        if (!pf_wait(&full_v[j % NST], (j / NST) & 1, abort, p.wait_ns)) break;
         tc_fence_after();
         issue_pv(0, j);
         const bool more = j + 1 < n_tiles;
         if (more) {
-          if (!pf_wait(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1, abort)) break;
+          if (!pf_wait(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1, abort, p.wait_ns)) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
         // tile B
-        if (!pf_wait(&p_full[1], j & 1, abort)) break;
+        if (!pf_wait(&p_full[1], j & 1, abort, p.wait_ns)) break;
         tc_fence_after();
         issue_pv(1, j);
         umma_commit(&empty[j % NST]);
         if (more) issue_s(1, j + 1);
       }
       umma_commit(drain);
-      mbar_wait_bounded(drain, 0, kPfWaitLimitNs);
+      mbar_wait_bounded(drain, 0, kPfDrainLimitNs);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -378,7 +384,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      ok = __all_sync(0xffffffffu, pf_wait(&s_full[x], j & 1, abort));
+      ok = __all_sync(0xffffffffu, pf_wait(&s_full[x], j & 1, abort, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
       // this half's 64 scores, read once (two loads) and kept in registers
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // overwritten by the next tile's)
       *slot(j & 1, half) = mr;
       mbar_arrive(pr_bar);
-      ok = __all_sync(0xffffffffu, pf_wait(pr_bar, j & 1, abort));
+      ok = __all_sync(0xffffffffu, pf_wait(pr_bar, j & 1, abort, p.wait_ns));
       if (!ok) break;
       mr = fmaxf(mr, *reinterpret_cast<volatile float *>(slot(j & 1, 1 - half)));
       // with a positive scale the maximum of the raw scores, scaled once
@@ -455,7 +461,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // O is stable once the previous P.V is done; rescale this half's
       // columns if the reference maximum moved
       if (j > 0) {
-        ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (j - 1) & 1, abort));
+        ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (j - 1) & 1, abort, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, bump)) {
@@ -480,7 +486,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // A's threads; tile B's P.V is issued after tile A's)
         const int z0 = pos_max + 1 - j * kPfKeys;
         if (z0 < kPfKeys) {
-          ok = __all_sync(0xffffffffu, pf_wait(&full_v[j % NST], (j / NST) & 1, abort));
+          ok = __all_sync(0xffffffffu, pf_wait(&full_v[j % NST], (j / NST) & 1, abort, p.wait_ns));
           if (!ok) break;
           const int tid = threadIdx.x - 64;
           uint8_t *v0 = sV + (j % NST) * L::KV_BYTES;
@@ -495,12 +501,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[x]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (n_tiles - 1) & 1, abort));
+    if (ok) ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (n_tiles - 1) & 1, abort, p.wait_ns));
     if (ok) {
       // the row sum: this half's plus the other half's (one more pair phase)
       *slot(2, half) = l;
       mbar_arrive(pr_bar);
-      ok = __all_sync(0xffffffffu, pf_wait(pr_bar, n_tiles & 1, abort));
+      ok = __all_sync(0xffffffffu, pf_wait(pr_bar, n_tiles & 1, abort, p.wait_ns));
     }
     if (ok) {
       tc_fence_after();

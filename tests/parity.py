@@ -19,9 +19,11 @@ TOL = 2e-3   # max-abs error allowed for attention outputs (fp32 accumulate vs f
 
 
 class Expected:
-    """Oracle result of one decode step on (a sample of) a generated batch."""
+    """Oracle result of one decode step on (a sample of) a generated batch.
+    With ``whole_pool`` the oracle's cache write is also applied to a host
+    copy of the entire pool (``k_pool``, ``v_pool``: bits after the step)."""
 
-    def __init__(self, batch: W.DecodeBatch, seqs=None):
+    def __init__(self, batch: W.DecodeBatch, seqs=None, whole_pool: bool = False):
         sh = batch.shape
         B = sh.block_size
         S = batch.num_seqs
@@ -34,6 +36,10 @@ class Expected:
             sl = bm.allocate(s, L)
             self.slots[s] = sl[-1] if L > 0 else -1
         self.tables = {s: bm.block_table(s) for s in range(S)}
+        if whole_pool:
+            self.k_pool, self.v_pool = W.bits(batch.k_cache), W.bits(batch.v_cache)
+            OC.reshape_and_cache(W.bits(batch.k_new), W.bits(batch.v_new), self.k_pool,
+                                 self.v_pool, self.slots, B)
         # the needed part of the pool, as drawn
         need = sorted({b for s in self.seqs for b in self.tables[s]})
         self.blocks = np.array(need, dtype=np.int64)
@@ -60,9 +66,11 @@ class Expected:
                                              sh.num_kv_heads, B, sh.dtype)
 
 
-def library_fused_step(pa, batch: W.DecodeBatch):
+def library_fused_step(pa, batch: W.DecodeBatch, max_context_len=None):
     """One decode step through the fused entry point pa_decode_step (cache
-    write of the newest token + attention in one launch).  Returns (tables, out)."""
+    write of the newest token + attention in one launch), with a workspace of
+    pa_paged_decode_workspace_bytes as the benchmark allocates it.  Returns
+    (tables, out)."""
     sh = batch.shape
     S = batch.num_seqs
     bm = pa.BlockManager(batch.num_blocks, sh.block_size, batch.free_order)
@@ -71,10 +79,14 @@ def library_fused_step(pa, batch: W.DecodeBatch):
     tables, lens = bm.block_tables(np.arange(S), batch.max_blocks_per_seq)
     dev = batch.q.device
     out = torch.empty(S, sh.num_q_heads, sh.head_dim, dtype=torch.float32, device=dev)
+    if max_context_len is None:
+        max_context_len = int(batch.context_lens.max(initial=0))
+    ws = pa.alloc_workspace(S, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, sh.block_size,
+                            max_context_len, dev)
     pa.pa_decode_step(out, batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache,
                       torch.as_tensor(tables, device=dev), torch.as_tensor(lens, device=dev),
-                      batch.scale, sh.num_kv_heads,
-                      max_context_len=int(batch.context_lens.max(initial=0)))
+                      batch.scale, sh.num_kv_heads, max_context_len=max_context_len,
+                      workspace=ws)
     torch.cuda.synchronize()
     return tables, out
 

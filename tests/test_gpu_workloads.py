@@ -1,7 +1,10 @@
 """GPU parity at full workload sizes, in the launch configuration the
-benchmark times: 13B-class, GQA 8B-class and long-context decode (sampled
-sequences, computed one by one by the oracle), and the 64-step parallel
-sampling run with copy-on-write (every step checked)."""
+benchmark times: 13B-class, GQA 8B-class and long-context decode, every
+sequence compared with the oracle and the whole pool compared bit for bit
+after the step's cache write, through both the fused entry point the
+benchmark times (pa_decode_step) and the two-call path (reshape_and_cache +
+paged decode attention); and the 64-step parallel sampling run with
+copy-on-write (every step checked)."""
 import numpy as np
 import pytest
 import torch
@@ -10,33 +13,32 @@ from oracle import attention as OA
 from oracle import cache_ops as OC
 from oracle.block_manager import BlockManager as OracleBM
 import workloads as W
-from parity import TOL, Expected, library_step, max_abs_err
+from parity import TOL, Expected, library_fused_step, library_step, max_abs_err
 
 pytestmark = pytest.mark.gpu
 
 
-def sample_seqs(lens, k, seed):
-    rng = np.random.default_rng(seed)
-    order = np.argsort(lens)
-    pick = {int(order[0]), int(order[-1]), int(order[len(order) // 2])}
-    pick |= set(int(x) for x in rng.choice(len(lens), size=min(k, len(lens)), replace=False))
-    return sorted(pick)
-
-
-@pytest.mark.parametrize("name,k", [("13b", 8), ("gqa8b", 12), ("long", 8), ("long32", 8)])
-def test_full_size_workload(pa, cuda_device, name, k):
+@pytest.mark.parametrize("name", ["13b", "gqa8b", "long", "long32"])
+@pytest.mark.parametrize("path", ["fused", "two_call"])
+def test_full_size_workload(pa, cuda_device, name, path):
     b = W.standard_batch(name, device=cuda_device)
-    seqs = sample_seqs(b.context_lens, k, 7)
-    exp = Expected(b, seqs)
-    slots, tables, out = library_step(pa, b)
-    assert np.array_equal(slots, exp.slots)
+    exp = Expected(b, whole_pool=True)          # every sequence, from the pool as drawn
+    if path == "fused":
+        # the benchmark's launch: pa_decode_step with a workspace sized for
+        # every tuning and the table's capacity as the context bound
+        tables, out = library_fused_step(pa, b, max_context_len=b.max_blocks_per_seq *
+                                         b.shape.block_size)
+    else:
+        slots, tables, out = library_step(pa, b)
+        assert np.array_equal(slots, exp.slots)
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        assert tables[s, :-(-L // b.shape.block_size)].tolist() == exp.tables[s]
     got = out.cpu().numpy()
-    err = max_abs_err(got[exp.seqs], exp.out)
+    err = max_abs_err(got, exp.out)
     assert err <= TOL, err
-    # every row is finite, and rows of unsampled sequences are softmax averages
-    # of V: within the range of the values drawn
-    assert np.isfinite(got).all()
-    assert np.abs(got).max() <= float(b.v_cache.abs().max()) + 1e-3
+    assert np.array_equal(W.bits(b.k_cache), exp.k_pool)
+    assert np.array_equal(W.bits(b.v_cache), exp.v_pool)
     assert pa.pa_device_error() == 0
 
 
