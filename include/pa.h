@@ -236,8 +236,10 @@ int pa_decode_tuning(int nstage, int ctas_per_sm, int min_tiles_per_warp);
  * has left) and returns; the output rows of that call are then undefined.
  * ns == 0 restores the default of 2 s, far above any copy's latency; a tiny
  * limit makes the waits run out on purpose, which is how failure detection
- * is tested without faulting or hanging the GPU.  Process-wide; returns
- * PA_ERR_ARG for ns < 0.  No counterpart on the pages.
+ * is tested without faulting or hanging the GPU.  Limits under 1 ms are
+ * polled (no sleeping wait) and counted in SM clock cycles at 2 per ns, so
+ * they run out no earlier than asked at clocks up to 2 GHz.  Process-wide;
+ * returns PA_ERR_ARG for ns < 0.  No counterpart on the pages.
  */
 int pa_set_wait_limit(long long ns);
 

@@ -69,30 +69,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait whose suspension lasts at most `hint_ns` (instead of the
-// hardware's own limit), so that a short wait limit can run out while the
-// awaited copy is still in flight.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity,
-                                                   uint32_t hint_ns) {
+// Non-blocking test of the barrier phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
 
-// Limits at or above this keep the plain try_wait (the normal case: 2 s).
+// Limits at or above this are timed with %globaltimer and use the blocking
+// try_wait (the normal case: 2 s).  Shorter ones -- set on purpose, to make
+// waits run out while copies are in flight -- poll with test_wait and are
+// timed in SM clock cycles, 2 per ns: the global timer advances in steps too
+// coarse for them, and try_wait may sleep until the copy has landed.
 constexpr uint64_t kShortWaitNs = 1000000ull;
 
-// One try_wait within a wait limited to `limit_ns`.
-__device__ __forceinline__ bool mbar_try_wait_within(uint64_t *bar, uint32_t parity,
-                                                     uint64_t limit_ns) {
-  if (limit_ns >= kShortWaitNs) return mbar_try_wait(bar, parity);
-  return mbar_try_wait_hint(bar, parity, (uint32_t)limit_ns);
+__device__ __forceinline__ bool mbar_wait_short(uint64_t *bar, uint32_t parity,
+                                                uint64_t limit_ns) {
+  const long long c0 = clock64();
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((uint64_t)(clock64() - c0) > 2 * limit_ns) return false;
+  }
 }
 
 // Wait for the barrier phase with the given parity to complete, giving up
@@ -100,10 +103,11 @@ __device__ __forceinline__ bool mbar_try_wait_within(uint64_t *bar, uint32_t par
 // PA_DEVERR_TIMEOUT and winds down).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns) {
-  if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
+  if (limit_ns < kShortWaitNs) return mbar_wait_short(bar, parity, limit_ns);
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }

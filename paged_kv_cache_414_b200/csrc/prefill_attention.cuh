@@ -97,17 +97,23 @@ struct PrefillSmem {
 // Bounded wait that also gives up when another role has aborted.
 __device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                         uint64_t limit_ns) {
-  if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait_within(bar, parity, limit_ns)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      *abort = 1;
-      flag_error(PA_DEVERR_TIMEOUT);
-      return false;
+  bool done;
+  if (limit_ns < kShortWaitNs) {            // a short limit set on purpose: poll, count cycles
+    const long long c0 = clock64();
+    while (!(done = mbar_test_wait(bar, parity)) && !*abort &&
+           (uint64_t)(clock64() - c0) <= 2 * limit_ns) {
     }
+  } else {
+    done = mbar_try_wait(bar, parity);
+    const uint64_t t0 = done ? 0 : globaltimer_ns();
+    while (!done && !*abort && globaltimer_ns() - t0 <= limit_ns) done = mbar_try_wait(bar, parity);
   }
+  if (done) return true;
+  if (!*abort) {
+    *abort = 1;
+    flag_error(PA_DEVERR_TIMEOUT);
+  }
+  return false;
 }
 
 // 2^x by the hardware approximation (ex2.approx, flush-to-zero); its error is
