@@ -318,26 +318,37 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint32_t idS = umma_idesc_f16(kBf, kPfRows, kPfKeys, false, false);
       const uint32_t idO = umma_idesc_f16(kBf, kPfRows, D, false, true);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+      // Shared-memory descriptors, built once: a k-step moves the start
+      // address field by a constant, so every MMA below takes a
+      // precomputed base plus an immediate (the issuing thread shares its
+      // scheduler with softmax warps, so its instruction count per MMA is
+      // what sets the issue rate).
+      const uint64_t dQ0 = umma_desc_sw128(aQ, 16, 1024);
+      const uint64_t dK0 = umma_desc_sw128(aK, 16, 1024);
+      const uint64_t dV0 = umma_desc_sw128(aV, kPfKeys * 128, 1024);
+      constexpr uint32_t kStageStep = L::KV_BYTES >> 4, kQStep = L::Q_TILE >> 4;
       auto issue_s = [&](int x, int j) {        // S_x = Q_x K_j^T
-        const uint32_t q = aQ + x * L::Q_TILE, k0 = aK + (j % NST) * L::KV_BYTES;
+        const uint64_t dq = dQ0 + x * kQStep, dk = dK0 + (j % NST) * kStageStep;
+        const uint32_t d = tmem + x * 256;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::REGION + (kk & 3) * 32;
-          umma_f16_ss(tmem + x * 256, umma_desc_sw128(q + off, 16, 1024),
-                      umma_desc_sw128(k0 + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          constexpr uint32_t kRegion = L::REGION >> 4;
+          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 2;
+          umma_f16_ss(d, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {       // O_x += P_x V_j
-        const uint32_t v0 = aV + (j % NST) * L::KV_BYTES, pj = tmem + x * 256;
+        const uint64_t dv = dV0 + (j % NST) * kStageStep;
+        const uint32_t pj = tmem + x * 256, d = pj + 128;
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kPfKeys / 16; ++kk) {
           // 16 keys: their 16 score columns hold 8 columns of hi weights, then
           // (bf16) 8 of lo weights; 16 rows of V
-          const uint64_t db = umma_desc_sw128(v0 + kk * 16 * 128, kPfKeys * 128, 1024);
-          const uint32_t pc = pj + kk * 16;
-          umma_f16_ts(tmem + x * 256 + 128, pc, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
-          if (PfPack<T>::kSplit) umma_f16_ts(tmem + x * 256 + 128, pc + 8, db, idO, 1u);
+          const uint64_t db = dv + kk * ((16 * 128) >> 4);
+          umma_f16_ts(d, pj + kk * 16, db, idO, kk > 0 ? 1u : acc0);
+          if (PfPack<T>::kSplit) umma_f16_ts(d, pj + kk * 16 + 8, db, idO, 1u);
         }
         umma_commit(&o_done[x]);
       };
@@ -393,28 +404,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       ok = __all_sync(0xffffffffu, pf_wait(&s_full[x], j & 1, abort, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
-      // this half's 64 scores, read once (two loads) and kept in registers
+      // this half's 64 scores: read for the maximum, then read again 32 at a
+      // time for the weights (keeping all 64 in registers costs spills)
       const uint32_t sj = tSx + half * 64;
       const int kh0 = j * kPfKeys + half * 64;   // first key of this half
       const bool diag = kh0 + 63 > pos_min;      // some key past some row's position
-      uint32_t v[64];
-      tmem_load32(sj, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_load32(sj + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      // pass 1: the maximum of the raw scores (masked on diagonal tiles)
       float mx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-      if (!pos_scale) {             // general scale: maximum of the scaled scores
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (kh0 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]) * sl2);
-      } else if (diag) {
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tmem_load32(sj + hh * 32, v);
+        if (!pos_scale) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (kh0 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
-      } else {
+          for (int i = 0; i < 32; ++i)
+            if (kh0 + hh * 32 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]) * sl2);
+        } else if (diag) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+          for (int i = 0; i < 32; ++i)
+            if (kh0 + hh * 32 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+        }
       }
       float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
@@ -440,14 +453,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // sum; per 16 keys, their 16 score columns take 8 columns of hi weights
       // and (bf16) 8 of lo weights; one wait for all the stores
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t v[32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        if ((c & 1) == 0) tmem_load32(sj + c * 16, v);
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int k = c * 16 + 2 * i;
-          float p0 = fast_exp2(fmaf(__uint_as_float(v[k]), sl2, -m_new));
-          float p1 = fast_exp2(fmaf(__uint_as_float(v[k + 1]), sl2, -m_new));
+          float p0 = fast_exp2(fmaf(__uint_as_float(v[k & 31]), sl2, -m_new));
+          float p1 = fast_exp2(fmaf(__uint_as_float(v[(k + 1) & 31]), sl2, -m_new));
           if (diag) {
             p0 = kh0 + k <= pos ? p0 : 0.f;
             p1 = kh0 + k + 1 <= pos ? p1 : 0.f;
