@@ -338,10 +338,10 @@ int launch_prefill(const PrefillArgs &a, int dev) {
   p.tq = tq;
   p.q_tiles = (a.max_query_len + 2 * tq - 1) / (2 * tq);   // a CTA takes two query tiles
   p.wait_ns = g_wait_limit_ns.load();
-  const long long nx = (long long)p.q_tiles * a.num_seqs;
+  const long long nx = (long long)p.q_tiles * a.num_seqs * a.num_kv_heads;
   if (nx >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)nx, (unsigned)a.num_kv_heads);
+  cfg.gridDim = dim3((unsigned)nx);   // (sequence by rank, query-tile pair, kv head)
   cfg.blockDim = dim3(pa::kPfThreads);
   cfg.dynamicSmemBytes = L::BYTES;
   cfg.stream = a.stream;

@@ -11,7 +11,8 @@
 // causally to positions 0 .. L_s - C_s + i:
 //   out[t, h] = softmax(scale * q[t, h] . K_s[0..p]) V_s[0..p].
 //
-// Work split: one CTA per (sequence, kv head, pair of query tiles).  A query
+// Work split: one CTA per (sequence, kv head, pair of query tiles), launched
+// longest sequence first (ranked in the kernel for up to 32 sequences).  A query
 // tile is 128 rows = TQ = 128 / G chunk tokens x the G query heads that share
 // the kv head; the CTA's two tiles (A, then B: 2 TQ consecutive tokens) share
 // every K/V tile fetched from the pool.  Keys go in tiles of 128 positions
@@ -55,6 +56,7 @@
 // bounded) and the tensor memory is freed.
 #pragma once
 
+#include <limits.h>
 #include <math.h>
 
 #include "umma.cuh"
@@ -182,7 +184,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
   uint64_t *full_k = bars + 0;     // [NST] K tile landed
   uint64_t *full_v = bars + 3;     // [NST] V tile landed
-  uint64_t *empty = bars + 6;      // [NST] K/V stage consumed by all four MMAs
+  uint64_t *empty_k = bars + 6;    // [NST] K tile consumed by both query tiles' S
+  uint64_t *empty_v = bars + 27;   // [NST] V tile consumed by both query tiles' P.V
   uint64_t *q_full = bars + 9;     // both Q tiles landed
   uint64_t *s_full = bars + 10;    // [query tile] S written
   uint64_t *p_full = bars + 12;    // [query tile] P written, O rescaled (256 arrivals)
@@ -194,12 +197,39 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   float *xch = reinterpret_cast<float *>(smem + L::OFF_X);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = blockIdx.x % p.num_seqs;
-  const int qt = p.q_tiles - 1 - blockIdx.x / p.num_seqs;   // longest tiles first
-  const int kh = blockIdx.y;
   const int G = p.group;
 
   grid_dependency_wait();     // the chunk's cache write may be the kernel before
+  // Work unit of this CTA: (sequence, pair of query tiles, kv head), the kv
+  // head varying fastest in launch order.  A unit's length is set by its
+  // sequence's context, so with up to 32 sequences they are ranked by
+  // context length (longest first, ties by index) and the launch order runs
+  // through them by rank: the longest units start first and the short ones
+  // fill the last wave.  More sequences keep the plain order (query-tile
+  // pair slowest), which balances about as well.
+  const int kh = blockIdx.x % p.num_kv_heads;
+  const int v = blockIdx.x / p.num_kv_heads;
+  int s, qt;
+  if (p.num_seqs <= 32) {
+    __shared__ int seq_of_rank;
+    const int rank_wanted = v / p.q_tiles;
+    qt = p.q_tiles - 1 - v % p.q_tiles;
+    if (warp == 0) {
+      const int Lm = lane < p.num_seqs ? __ldg(p.context_lens + lane) : INT_MIN;
+      int rank = 0;
+      for (int k = 0; k < p.num_seqs; ++k) {
+        const int Lk = __shfl_sync(0xffffffffu, Lm, k);
+        rank += (Lk > Lm || (Lk == Lm && k < lane)) ? 1 : 0;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, lane < p.num_seqs && rank == rank_wanted);
+      if (lane == 0) seq_of_rank = __ffs(hit) - 1;
+    }
+    __syncthreads();
+    s = seq_of_rank;
+  } else {
+    s = v % p.num_seqs;
+    qt = p.q_tiles - 1 - v / p.num_seqs;
+  }
   const int q0 = __ldg(p.query_start + s);
   const int C = __ldg(p.query_start + s + 1) - q0;
   const int Lc = __ldg(p.context_lens + s);
@@ -223,7 +253,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full_k[i], 1);
       mbar_init(&full_v[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty_k[i], 1);
+      mbar_init(&empty_v[i], 1);
     }
     mbar_init(q_full, 1);
     for (int x = 0; x < 2; ++x) {
@@ -273,7 +304,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks;
-    int issued = 0;
+    // K and V of a stage are released separately: K as soon as both query
+    // tiles' S of its tile ran, V after their P.V, so the next K load starts
+    // about one tile earlier than a joint release would allow.
+    int issued_k = 0, issued_v = 0;
     for (int j = 0; j < n_tiles; ++j) {
       const int st = j % NST;
       // this lane's block id, fetched before the stage is free
@@ -285,30 +319,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (v >= 0 && v < p.num_blocks) id = v; else bad = true;
       }
       if (bad && cc == 0 && ckv == 0) flag_error(PA_DEVERR_BLOCK_ID);
+      const unsigned valid = __ballot_sync(0xffffffffu, id >= 0);
+      const int off = st * L::KV_BYTES + cc * kPfKeys * 128 + cb * B * 128;
+      const int row = (id * p.num_kv_heads + kh) * B;
       if (j >= NST) {
-        const bool w = lane == 0 ? pf_wait(&empty[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
+        const bool w = lane == 0 ? pf_wait(&empty_k[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
         if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
-      const unsigned valid = __ballot_sync(0xffffffffu, id >= 0);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full_k[st], __popc(valid & 0x55555555u) * B * 128);
-        mbar_arrive_expect_tx(&full_v[st], __popc(valid & 0xAAAAAAAAu) * B * 128);
-      }
+      if (lane == 0) mbar_arrive_expect_tx(&full_k[st], __popc(valid & 0x55555555u) * B * 128);
       __syncwarp();
-      if (id >= 0) {
-        const int off = st * L::KV_BYTES + cc * kPfKeys * 128 + cb * B * 128;
-        const int row = (id * p.num_kv_heads + kh) * B;
-        if (ckv == 0) tma_load_2d(sK + off, &kmap, cc * 64, row, &full_k[st]);
-        else tma_load_2d(sV + off, &vmap, cc * 64, row, &full_v[st]);
+      if (id >= 0 && ckv == 0) tma_load_2d(sK + off, &kmap, cc * 64, row, &full_k[st]);
+      issued_k = j + 1;
+      if (j >= NST) {
+        const bool w = lane == 0 ? pf_wait(&empty_v[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
+        if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
-      issued = j + 1;
+      if (lane == 0) mbar_arrive_expect_tx(&full_v[st], __popc(valid & 0xAAAAAAAAu) * B * 128);
+      __syncwarp();
+      if (id >= 0 && ckv == 1) tma_load_2d(sV + off, &vmap, cc * 64, row, &full_v[st]);
+      issued_v = j + 1;
     }
     // copies still in flight must land before the CTA exits
     if (lane == 0) {
-      for (int j = max(0, issued - NST); j < issued; ++j) {
+      for (int j = max(0, issued_k - NST); j < issued_k; ++j)
         mbar_wait_bounded(&full_k[j % NST], (j / NST) & 1, kPfDrainLimitNs);
+      for (int j = max(0, issued_v - NST); j < issued_v; ++j)
         mbar_wait_bounded(&full_v[j % NST], (j / NST) & 1, kPfDrainLimitNs);
-      }
       mbar_wait_bounded(q_full, 0, kPfDrainLimitNs);
     }
   } else if (warp == 1) {
@@ -357,6 +393,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
+        umma_commit(&empty_k[0]);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         // tile A: its P.V, then its next S (which overwrites its P, in issue order)
@@ -374,8 +411,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!pf_wait(&p_full[1], j & 1, abort, p.wait_ns)) break;
         tc_fence_after();
         issue_pv(1, j);
-        umma_commit(&empty[j % NST]);
-        if (more) issue_s(1, j + 1);
+        umma_commit(&empty_v[j % NST]);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(&empty_k[(j + 1) % NST]);
+        }
       }
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, kPfDrainLimitNs);
@@ -516,9 +556,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             *reinterpret_cast<uint4 *>(v0 + c * kPfKeys * 128 + (z0 + rem / 8) * 128 +
                                        (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
           }
+          // the zeros are written by this (generic) proxy and read by the
+          // tensor cores (async proxy): order them before the arrival
+          fence_proxy_async_smem();
         }
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[x]);
     }
