@@ -293,6 +293,21 @@ bool encode_query_map(CUtensorMap *m, const void *q, int T, int Hq, int D, int G
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// out [T, Hq, D] fp32 as a 3-D map (D, Hq, T) for the prefill epilogue's TMA
+// stores: a box is 32 columns x the G heads of one kv head x TQ tokens,
+// 128-byte swizzled in shared memory.
+bool encode_out_map(CUtensorMap *m, float *out, int T, int Hq, int D, int G, int tq) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)Hq * D * 4};
+  cuuint32_t box[3] = {32u, (cuuint32_t)G, (cuuint32_t)tq};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct PrefillArgs {
   float *out;
   const void *q, *k_cache, *v_cache;
@@ -316,11 +331,12 @@ int launch_prefill(const PrefillArgs &a, int dev) {
   }
   const int G = a.num_q_heads / a.num_kv_heads;
   const int tq = pa::kPfRows / G;
-  CUtensorMap qmap, kmap, vmap;
+  CUtensorMap qmap, kmap, vmap, omap;
   const long long rows = (long long)a.num_blocks * a.num_kv_heads * B;
   if (!encode_query_map(&qmap, a.q, a.num_tokens, a.num_q_heads, D, G, tq) ||
       !encode_pool_map(&kmap, a.k_cache, rows, D, B) ||
-      !encode_pool_map(&vmap, a.v_cache, rows, D, B))
+      !encode_pool_map(&vmap, a.v_cache, rows, D, B) ||
+      !encode_out_map(&omap, a.out, a.num_tokens, a.num_q_heads, D, G, tq))
     return PA_ERR_CUDA;
   pa::PrefillParams p;
   p.out = a.out;
@@ -350,7 +366,7 @@ int launch_prefill(const PrefillArgs &a, int dev) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, qmap, kmap, vmap, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, qmap, kmap, vmap, omap, p) != cudaSuccess) {
     cudaGetLastError();
     return PA_ERR_CUDA;
   }

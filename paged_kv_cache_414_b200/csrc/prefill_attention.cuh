@@ -170,7 +170,8 @@ template <typename T, int D, int B>
 __global__ void __launch_bounds__(kPfThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                          const __grid_constant__ CUtensorMap kmap,
-                         const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
+                         const __grid_constant__ CUtensorMap vmap,
+                         const __grid_constant__ CUtensorMap omap, const PrefillParams p) {
   using L = PrefillSmem<D>;
   constexpr int NCH = L::NCH;
   constexpr int NST = L::STAGES;
@@ -571,6 +572,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_arrive(pr_bar);
       ok = __all_sync(0xffffffffu, pf_wait(pr_bar, n_tiles & 1, abort, p.wait_ns));
     }
+    // Epilogue: out = O / l.  A tile whose rows all belong to the chunk goes
+    // through shared memory -- this tile's now idle ring (K for tile A, V for
+    // tile B: every MMA that read it has completed once o_done arrived) -- in
+    // the 128-byte-swizzled layout of the output tensor map, then out as TMA
+    // stores of 32-column boxes, so each row is written with whole lines
+    // instead of a 512-byte stride between lanes.  The last tile of a chunk,
+    // which may end inside it, is stored row by row.
+    const bool full_tile = tokx + p.tq <= C;
+    uint8_t *ostage = x == 0 ? sK : sV;
+    constexpr int OBOX = kPfRows * 128;           // one 32-column box of 128 rows
     if (ok) {
       tc_fence_after();
       l += *reinterpret_cast<volatile float *>(slot(2, 1 - half));
@@ -581,13 +592,33 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t o[16];
         tmem_load16(tOx + half * (D / 2) + c4 * 16, o);
-        if (row_ok) {
+        const int col0 = half * (D / 2) + c4 * 16;     // first of these 16 columns
+        uint8_t *box = ostage + (col0 >> 5) * OBOX + r * 128;
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4 *>(dst + c4 * 16 + i) =
-                make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                            __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+        for (int i = 0; i < 16; i += 4) {
+          const float4 val =
+              make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                          __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          if (full_tile) {
+            const int chunk = ((col0 & 31) + i) >> 2;   // 16-byte chunk within the box row
+            *reinterpret_cast<float4 *>(box + ((chunk ^ (r & 7)) << 4)) = val;
+          } else if (row_ok) {
+            *reinterpret_cast<float4 *>(dst + c4 * 16 + i) = val;
+          }
         }
+      }
+    }
+    if (full_tile) {
+      // every thread of the tile reaches this barrier, whether or not it
+      // aborted: the branch above holds no early exit
+      fence_proxy_async_smem();
+      named_barrier_sync(1 + x, 256);
+      if (warp == 2 + 8 * x && lane == 0 && !*abort) {
+#pragma unroll 1
+        for (int b = 0; b < D / 32; ++b)
+          tma_store_3d(&omap, ostage + b * OBOX, b * 32, kh * G, q0 + tokx);
+        bulk_commit_group();
+        bulk_wait_group0();
       }
     }
   }
