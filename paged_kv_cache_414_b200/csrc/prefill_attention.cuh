@@ -126,6 +126,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed pairs of fp32 lanes (one instruction for two values): (a0, a1) * b + c
+// and a + b on the pairs.
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0,
+                                      float b1, float c0, float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float &d0, float &d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fsub2(float &d0, float &d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Rounding of the softmax weights to the MMA's input type.
 template <typename T>
 struct PfPack;
@@ -140,8 +167,8 @@ struct PfPack<__nv_bfloat16> {
   __device__ __forceinline__ static void split2(float a, float b, uint32_t *hi, uint32_t *lo) {
     const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
     *hi = __byte_perm(ua, ub, 0x7632);
-    const float ra = a - __uint_as_float(ua & 0xffff0000u);
-    const float rb = b - __uint_as_float(ub & 0xffff0000u);
+    float ra, rb;
+    fsub2(ra, rb, a, b, __uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u));
     *lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
   }
   __device__ __forceinline__ static uint32_t round2(float a, float b, float *sum) {
@@ -493,6 +520,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, partial row
       // sum; per 16 keys, their 16 score columns take 8 columns of hi weights
       // and (bf16) 8 of lo weights; one wait for all the stores
+      // (pairs of keys use packed two-lane fp32 instructions)
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t v[32];
 #pragma unroll
@@ -502,15 +530,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int k = c * 16 + 2 * i;
-          float p0 = fast_exp2(fmaf(__uint_as_float(v[k & 31]), sl2, -m_new));
-          float p1 = fast_exp2(fmaf(__uint_as_float(v[(k + 1) & 31]), sl2, -m_new));
+          float x0, x1;
+          ffma2(x0, x1, __uint_as_float(v[k & 31]), __uint_as_float(v[(k + 1) & 31]), sl2, sl2,
+                -m_new, -m_new);
+          float p0 = fast_exp2(x0);
+          float p1 = fast_exp2(x1);
           if (diag) {
             p0 = kh0 + k <= pos ? p0 : 0.f;
             p1 = kh0 + k + 1 <= pos ? p1 : 0.f;
           }
           if (PfPack<T>::kSplit) {
             PfPack<T>::split2(p0, p1, &hi[i], &lo[i]);
-            sum[i & 3] += p0 + p1;
+            fadd2(sum[(i & 1) * 2], sum[(i & 1) * 2 + 1], sum[(i & 1) * 2], sum[(i & 1) * 2 + 1],
+                  p0, p1);
           } else {
             hi[i] = PfPack<T>::round2(p0, p1, &sum[i & 3]);
           }
