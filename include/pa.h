@@ -74,6 +74,8 @@ typedef enum {
 #define PA_DEVERR_SLOT 0x4u        /* slot_mapping entry >= num_blocks * block_size */
 #define PA_DEVERR_COPY_PAIR 0x8u   /* copy_blocks pair outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x10u    /* a bounded wait on an asynchronous copy gave up */
+#define PA_DEVERR_RANGE 0x20u      /* prefill: a bf16 V value beyond fp16's range (|v| > 65504,
+                                      or not finite) was saturated */
 
 /* Human-readable name of a pa_status value (static string). */
 const char *pa_status_string(int status);
@@ -286,10 +288,13 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
  *                longer chunk past what the grid covers are not computed, and
  *                PA_DEVERR_CONTEXT_LEN is set)
  * head_dim 64 or 128, block_size 16 or 32, group size up to 16, fp16 or
- * bf16.  Runs on the tensor cores (tcgen05, fp32 accumulation): the softmax
- * weights P enter P.V in the cache dtype -- for bf16 as a hi + lo pair of
- * bf16 values (relative error under 2^-14 per weight), for fp16 as one fp16
- * value (2^-11).  No workspace, nothing allocated.  A chunk longer than its
+ * bf16.  Runs on the tensor cores (tcgen05, fp32 accumulation): Q.K^T in the
+ * cache dtype; P.V in fp16 -- the softmax weights rounded to fp16 (2^-11
+ * relative; the row sums add the rounded values), and a bf16 V tile converted
+ * to fp16 in shared memory, which is exact for |v| <= 65504.  A bf16 V value
+ * beyond that (or not finite) is saturated to fp16's largest value and sets
+ * PA_DEVERR_RANGE: the rows attending to it are then inexact.  No workspace,
+ * nothing allocated.  A chunk longer than its
  * context, a context longer than the table, or rows outside
  * [0, num_tokens) set PA_DEVERR_CONTEXT_LEN and leave that sequence's rows
  * unwritten; block ids outside the pool are skipped and set

@@ -26,7 +26,8 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 PA_F16, PA_BF16 = 0, 1
 STATUS = {0: "PA_OK", -1: "PA_ERR_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_NO_BLOCKS",
           -4: "PA_ERR_SEQ", -5: "PA_ERR_CUDA", -6: "PA_ERR_DEVICE_BOUNDS", -7: "PA_ERR_WORKSPACE"}
-DEVERR = {"block_id": 0x1, "context_len": 0x2, "slot": 0x4, "copy_pair": 0x8, "timeout": 0x10}
+DEVERR = {"block_id": 0x1, "context_len": 0x2, "slot": 0x4, "copy_pair": 0x8, "timeout": 0x10,
+          "range": 0x20}
 
 
 class PAError(RuntimeError):

@@ -21,12 +21,13 @@
 //
 //   warp 0      TMA producer: both Q tiles once, then K/V tiles into a ring;
 //               each lane issues one copy of a tile (one block, one 64-column
-//               chunk, K or V), and K and V land on separate barriers.
+//               chunk, K or V), and K and V land on separate barriers; K and V
+//               of a stage are released separately.
 //   warp 1      owns the tensor memory; one lane issues the MMAs, alternating
 //               between the query tiles so that one tile's MMAs run while the
 //               other tile's softmax does:
-//                 S_X = Q_X K_j^T   (M 128, N 128 keys, K = head_dim)
-//                 O_X += P_X V_j    (M 128, N = head_dim, K 128 keys)
+//                 S_X = Q_X K_j^T   (M 128, N 128 keys, K = head_dim, cache dtype)
+//                 O_X += P_X V_j    (M 128, N = head_dim, K 128 keys, fp16)
 //               in the order S_A(0) S_B(0), then per tile j: O_A += P_A V_j,
 //               S_A(j+1), O_B += P_B V_j, S_B(j+1).
 //   warps 2-9   softmax of tile A, warps 10-17 of tile B, two threads per
@@ -35,21 +36,26 @@
 //               tile (through shared memory, ordered by a 64-arrival mbarrier
 //               per pair and the same bounded wait as everything else) and
 //               partial sums once at the end.  Online maximum and sum in
-//               fp32; the weights go to tensor memory, where the P.V MMA reads
-//               them as its A operand.  For bf16, P = P_hi + P_lo (both bf16, two
-//               MMAs, each cut from the fp32 weight by bit operations), so P
-//               carries under 2^-14 relative error instead of bf16's 2^-9;
-//               for fp16 one fp16 P whose rounded weights are
-//               also what the sum adds.  O is rescaled in tensor memory when
-//               the row maximum moves by more than 2^8; the epilogue writes
-//               out = O / l.
+//               fp32; the weights go to tensor memory as fp16 (the row sums
+//               add the rounded values, so the normalisation matches what the
+//               MMA multiplies), where the P.V MMA reads them as its A operand.
+//               O is rescaled in tensor memory when the row maximum moves by
+//               more than 2^8; the epilogue writes out = O / l, full query
+//               tiles through shared memory and TMA stores.
+//   warps 18-21 V converter: zero the rows of a V tile past the last visible
+//               key and, for bf16 caches, rewrite the tile in place as fp16
+//               (exact for |v| <= 65504; saturated beyond, with
+//               PA_DEVERR_RANGE), so P.V is one fp16 MMA per 16 keys.  The
+//               conversion sits between a V tile's arrival and its P.V, so
+//               it gets four warps (at 704 threads every thread keeps 80
+//               registers: the softmax re-reads its scores from TMEM rather
+//               than holding them).
 //
 // Tensor memory (512 columns): tile A's S at 0 and O at 128, tile B's S at
 // 256 and O at 384.  P replaces S in its own columns, 16 keys at a time: the
-// 16 columns holding those keys' scores take their 8 columns of hi weights
-// (two per column) and, for bf16, 8 of lo weights.  The MMA that next writes
-// a tile's S columns is issued after that tile's P.V, and MMAs run in issue
-// order.
+// 16 columns holding those keys' scores take their 8 columns of fp16 weights
+// (two per column).  The MMA that next writes a tile's S columns is issued
+// after that tile's P.V, and MMAs run in issue order.
 //
 // Every wait is bounded: on time-out a shared abort flag stops every role,
 // PA_DEVERR_TIMEOUT is set, copies and MMAs in flight are waited for (again
@@ -58,6 +64,8 @@
 
 #include <limits.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "umma.cuh"
 
@@ -77,7 +85,7 @@ struct PrefillParams {
 
 constexpr int kPfRows = 128;      // query rows per query tile
 constexpr int kPfKeys = 128;      // keys per K/V tile
-constexpr int kPfThreads = 576;   // producer warp, MMA warp, 2 x 8 softmax warps
+constexpr int kPfThreads = 704;   // producer, MMA, 2 x 8 softmax warps, 4 V-converter warps
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint64_t kPfDrainLimitNs = 2000000000ull;   // draining after an abort
 
@@ -92,7 +100,7 @@ struct PrefillSmem {
   static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  static constexpr int OFF_X = OFF_BAR + 256;         // pair exchange: [tile][set][half][row]
+  static constexpr int OFF_X = OFF_BAR + 512;         // pair exchange: [tile][set][half][row]
   static constexpr int BYTES = OFF_X + 2 * 3 * 2 * 128 * 4 + 1024;  // + alignment slack
 };
 
@@ -126,6 +134,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Packed pairs of fp32 lanes (one instruction for two values): (a0, a1) * b + c
 // and a + b on the pairs.
 __device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0,
@@ -153,45 +168,26 @@ __device__ __forceinline__ void fsub2(float &d0, float &d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// Rounding of the softmax weights to the MMA's input type.
-template <typename T>
-struct PfPack;
-template <>
-struct PfPack<__nv_bfloat16> {
-  static constexpr bool kBf16 = true;
-  static constexpr bool kSplit = true;     // P = hi + lo
-  // (a, b) -> packed hi pair, packed lo pair.  hi is each weight cut to bf16
-  // (its upper 16 bits), lo the exact remainder cut to bf16 the same way, so
-  // hi + lo is the weight within 2^-14 relative; bit operations and fp32
-  // subtractions only, no conversion instructions.
-  __device__ __forceinline__ static void split2(float a, float b, uint32_t *hi, uint32_t *lo) {
-    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
-    *hi = __byte_perm(ua, ub, 0x7632);
-    float ra, rb;
-    fsub2(ra, rb, a, b, __uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u));
-    *lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
-  }
-  __device__ __forceinline__ static uint32_t round2(float a, float b, float *sum) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    float2 f = __bfloat1622float2(h);
-    *sum += f.x + f.y;
-    return *reinterpret_cast<uint32_t *>(&h);
-  }
-};
-template <>
-struct PfPack<__half> {
-  static constexpr bool kBf16 = false;
-  static constexpr bool kSplit = false;    // one fp16 P
-  __device__ __forceinline__ static void split2(float, float, uint32_t *, uint32_t *) {}
-  // round two weights to fp16; return the packed pair and add the rounded
-  // values to *sum (so the normalisation matches what the MMA multiplies)
-  __device__ __forceinline__ static uint32_t round2(float a, float b, float *sum) {
-    __half2 h = __floats2half2_rn(a, b);
-    float2 f = __half22float2(h);
-    *sum += f.x + f.y;
-    return *reinterpret_cast<uint32_t *>(&h);
-  }
-};
+// A packed pair of bf16 values as a packed pair of fp16 values: exact within
+// fp16's range (bf16 has fewer significant bits), saturating beyond it; *big
+// keeps the largest magnitude seen.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x, float *big) {
+  const float hi = __uint_as_float(x & 0xffff0000u), lo = __uint_as_float(x << 16);
+  *big = fmax3(*big, fabsf(hi), fabsf(lo));
+  uint32_t y;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
+// Two weights rounded to fp16 (packed, the first in the low half); the
+// rounded values are what the row sums add, so the normalisation matches
+// what the MMA multiplies.
+__device__ __forceinline__ uint32_t round_f16(float a, float b, float *s0, float *s1) {
+  __half2 h = __floats2half2_rn(a, b);
+  const float2 f = __half22float2(h);
+  fadd2(*s0, *s1, *s0, *s1, f.x, f.y);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
 
 template <typename T, int D, int B>
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -222,6 +218,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t *pair = bars + 17;      // [query tile][row quarter] the two threads of a row
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
   volatile int *abort = reinterpret_cast<volatile int *>(bars + 26);
+  uint64_t *v_ready = bars + 32;   // [NST] V tile in fp16 with its tail zeroed
+
   float *xch = reinterpret_cast<float *>(smem + L::OFF_X);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -283,7 +281,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&full_v[i], 1);
       mbar_init(&empty_k[i], 1);
       mbar_init(&empty_v[i], 1);
+      mbar_init(&v_ready[i], 128);
     }
+
     mbar_init(q_full, 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
@@ -378,9 +378,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      constexpr bool kBf = PfPack<T>::kBf16;
+      constexpr bool kBf = std::is_same<T, __nv_bfloat16>::value;
       const uint32_t idS = umma_idesc_f16(kBf, kPfRows, kPfKeys, false, false);
-      const uint32_t idO = umma_idesc_f16(kBf, kPfRows, D, false, true);
+      const uint32_t idO16 = umma_idesc_f16(false, kPfRows, D, false, true);   // fp16 P and V
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
       // Shared-memory descriptors, built once: a k-step moves the start
       // address field by a constant, so every MMA below takes a
@@ -402,18 +402,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         umma_commit(&s_full[x]);
       };
-      auto issue_pv = [&](int x, int j) {       // O_x += P_x V_j
+      auto issue_pv = [&](int x, int j) {       // O_x += P_x V_j, fp16 P and V
         const uint64_t dv = dV0 + (j % NST) * kStageStep;
         const uint32_t pj = tmem + x * 256, d = pj + 128;
         const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kPfKeys / 16; ++kk) {
-          // 16 keys: their 16 score columns hold 8 columns of hi weights, then
-          // (bf16) 8 of lo weights; 16 rows of V
-          const uint64_t db = dv + kk * ((16 * 128) >> 4);
-          umma_f16_ts(d, pj + kk * 16, db, idO, kk > 0 ? 1u : acc0);
-          if (PfPack<T>::kSplit) umma_f16_ts(d, pj + kk * 16 + 8, db, idO, 1u);
-        }
+        for (int kk = 0; kk < kPfKeys / 16; ++kk)   // 16 keys: 8 columns of P, 16 rows of V
+          umma_f16_ts(d, pj + kk * 16, dv + kk * ((16 * 128) >> 4), idO16, kk > 0 ? 1u : acc0);
         umma_commit(&o_done[x]);
       };
       bool ok = pf_wait(q_full, 0, abort, p.wait_ns) && pf_wait(&full_k[0], 0, abort, p.wait_ns);
@@ -426,7 +421,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int j = 0; ok && j < n_tiles; ++j) {
         // tile A: its P.V, then its next S (which overwrites its P, in issue order)
         if (!pf_wait(&p_full[0], j & 1, abort, p.wait_ns)) break;
-        if (!pf_wait(&full_v[j % NST], (j / NST) & 1, abort, p.wait_ns)) break;
+        if (!pf_wait(&v_ready[j % NST], (j / NST) & 1, abort, p.wait_ns)) break;
         tc_fence_after();
         issue_pv(0, j);
         const bool more = j + 1 < n_tiles;
@@ -448,6 +443,39 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, kPfDrainLimitNs);
     }
+  } else if (warp >= 18) {
+    // ------------------------------------------------------------ V converter
+    // Each landed V tile, before its P.V: rows past the last visible key are
+    // zeroed (masked for every row, but 0 x NaN from stale or poisoned bits
+    // would reach O), and a bf16 tile is rewritten in place as fp16 -- exact
+    // for |v| <= 65504, fp16's largest value; beyond it the value saturates
+    // there and PA_DEVERR_RANGE is set -- so that P.V takes one fp16 P.  An
+    // element keeps its byte position, so the swizzle is untouched.
+    const int ct = threadIdx.x - 18 * 32;          // 0 .. 127
+    constexpr int NCHUNK = NCH * kPfKeys * 8;      // 16-byte chunks of a V tile
+    constexpr bool kBf = std::is_same<T, __nv_bfloat16>::value;
+    float big = 0.f;                               // largest |v| of the bf16 values kept
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j % NST;
+      if (!__all_sync(0xffffffffu, pf_wait(&full_v[st], (j / NST) & 1, abort, p.wait_ns)))
+        break;
+      uint8_t *v0 = sV + st * L::KV_BYTES;
+      const int z0 = j == n_tiles - 1 ? pos_max + 1 - j * kPfKeys : kPfKeys;   // first dead row
+      for (int i = ct; i < NCHUNK; i += 128) {
+        uint4 *c = reinterpret_cast<uint4 *>(v0 + i * 16);
+        if (((i >> 3) & (kPfKeys - 1)) >= z0) {
+          *c = make_uint4(0, 0, 0, 0);
+        } else if (kBf) {
+          const uint4 w = *c;
+          *c = make_uint4(bf16x2_to_f16x2(w.x, &big), bf16x2_to_f16x2(w.y, &big),
+                          bf16x2_to_f16x2(w.z, &big), bf16x2_to_f16x2(w.w, &big));
+        }
+      }
+      // generic-proxy writes, read next by the tensor cores (async proxy)
+      fence_proxy_async_smem();
+      mbar_arrive(&v_ready[st]);
+    }
+    if (kBf && !(big <= 65504.f)) flag_error(PA_DEVERR_RANGE);   // beyond fp16, or infinite
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int x = (warp - 2) >> 3;                // query tile: warps 2-9 A, 10-17 B
@@ -494,7 +522,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (kh0 + hh * 32 + i <= pos) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+          for (int i = 0; i < 16; ++i)
+            mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
       }
       float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -526,7 +555,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         if ((c & 1) == 0) tmem_load32(sj + c * 16, v);
-        uint32_t hi[8], lo[8];
+        uint32_t hp[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int k = c * 16 + 2 * i;
@@ -539,16 +568,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             p0 = kh0 + k <= pos ? p0 : 0.f;
             p1 = kh0 + k + 1 <= pos ? p1 : 0.f;
           }
-          if (PfPack<T>::kSplit) {
-            PfPack<T>::split2(p0, p1, &hi[i], &lo[i]);
-            fadd2(sum[(i & 1) * 2], sum[(i & 1) * 2 + 1], sum[(i & 1) * 2], sum[(i & 1) * 2 + 1],
-                  p0, p1);
-          } else {
-            hi[i] = PfPack<T>::round2(p0, p1, &sum[i & 3]);
-          }
+          hp[i] = round_f16(p0, p1, &sum[(i & 1) * 2], &sum[(i & 1) * 2 + 1]);
         }
-        tmem_store8_async(sj + c * 16, hi);
-        if (PfPack<T>::kSplit) tmem_store8_async(sj + c * 16 + 8, lo);
+        tmem_store8_async(sj + c * 16, hp);
       }
       tmem_store_wait();
       l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
@@ -572,26 +594,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[8 + i]) * alpha);
             tmem_store8(oc + 8, o8);
           }
-        }
-      }
-      if (x == 0 && j == n_tiles - 1) {
-        // keys past pos_max are masked for every row; their V rows may hold
-        // stale or poisoned bits, and 0 * NaN would reach O: zero them (tile
-        // A's threads; tile B's P.V is issued after tile A's)
-        const int z0 = pos_max + 1 - j * kPfKeys;
-        if (z0 < kPfKeys) {
-          ok = __all_sync(0xffffffffu, pf_wait(&full_v[j % NST], (j / NST) & 1, abort, p.wait_ns));
-          if (!ok) break;
-          const int tid = threadIdx.x - 64;
-          uint8_t *v0 = sV + (j % NST) * L::KV_BYTES;
-          for (int i = tid; i < NCH * (kPfKeys - z0) * 8; i += 256) {
-            const int c = i / ((kPfKeys - z0) * 8), rem = i % ((kPfKeys - z0) * 8);
-            *reinterpret_cast<uint4 *>(v0 + c * kPfKeys * 128 + (z0 + rem / 8) * 128 +
-                                       (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
-          }
-          // the zeros are written by this (generic) proxy and read by the
-          // tensor cores (async proxy): order them before the arrival
-          fence_proxy_async_smem();
         }
       }
       tc_fence_before();

@@ -199,3 +199,18 @@ def test_bad_block_id_reports_instead_of_faulting(pa, cuda_device):
     rows = np.arange(b.query_start[1], b.query_start[2])
     assert max_abs_err(out.cpu().numpy()[rows], want[rows]) <= TOL
     assert pa.pa_device_error() == 0
+
+
+def test_bf16_values_beyond_fp16_range_are_reported(pa, cuda_device):
+    """P.V runs in fp16, with a bf16 V tile converted exactly within fp16's
+    range; a bf16 V value beyond it is saturated and reported
+    (PA_DEVERR_RANGE), never silent.  Sequences that never read the value
+    still match the oracle."""
+    sh = W.Shape(8, 2, 128, 16, "bf16")
+    b = W.make_prefill_batch(sh, [300, 500], [100, 200], seed=9, device=cuda_device)
+    blk = int(b.block_tables[1, 0])                  # a prefix block of sequence 1
+    b.v_cache[blk, 0, 3, 5] = 1.0e6
+    got, want = run_prefill(pa, b)
+    assert pa.pa_device_error() == pa.DEVERR["range"]
+    rows0 = slice(int(b.query_start[0]), int(b.query_start[1]))
+    assert max_abs_err(got[rows0], want[rows0]) <= TOL
