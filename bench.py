@@ -86,7 +86,7 @@ PREFILL_PROFILE = os.path.join(ROOT, "profiles", "prefill_attention_16x512.md")
 PREFILL_SOURCES = ["paged_kv_cache_414_b200/csrc/prefill_attention.cuh",
                    "paged_kv_cache_414_b200/csrc/umma.cuh",
                    "paged_kv_cache_414_b200/csrc/pa_device.cuh",
-                   "paged_kv_cache_414_b200/csrc/pa_kernels.cu"]
+                   "paged_kv_cache_414_b200/csrc/prefill_launch.cuh"]
 
 
 def kernel_source_sha(sources=None) -> str:
