@@ -831,8 +831,8 @@ def run_prefill_b200(args, rank, world, local_rank):
                                 "workload (profiles/prefill_attention_16x512.md)",
                 "flops_per_launch": pb.flops,
                 "flops_note": "algorithmic: 4*D*Hq*(p+1) per chunk token; the kernel also "
-                              "multiplies the masked half of diagonal tiles and, for bf16, "
-                              "P.V twice (hi + lo weights), which are not counted",
+                              "multiplies the masked part of diagonal tiles, which is not "
+                              "counted",
                 "avg_launch_ms": round(attn_ms, 5),
                 "launch_timing": "CUDA events around every prefill call",
             },
