@@ -261,6 +261,7 @@ class Workload:
         import torch
         self.name = name
         self.cyclic = False
+        self.steps_total = steps_total   # the block tables are sized for this many steps
         if name == "cow":
             self._init_cow(device, seed_offset, steps_total)
             return
@@ -1133,7 +1134,7 @@ def cpu_baseline(wl, seconds: float):
     sequences until about `seconds` of CPU work are spent."""
     rng = np.random.default_rng(0)
     spent, nbytes, done, step = 0.0, 0, 0, 0
-    while spent < seconds and step < 64:
+    while spent < seconds and step < wl.steps_total:
         for s in rng.permutation(wl.S):
             dt, nb = oracle_step_sample(wl, step, [int(s)])
             spent += dt
