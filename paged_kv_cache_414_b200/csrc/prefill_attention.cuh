@@ -546,6 +546,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const float m_new = bump ? mt : m;
       const float alpha = bump ? fast_exp2(m - m_new) : 1.f;
       m = m_new;
+      // Rescale this half's columns of O if the reference maximum moved.  O
+      // is stable: S(j) was committed after P.V(j-1), and its arrival is what
+      // this tile started on.
+      if (j > 0 && __any_sync(0xffffffffu, bump)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 2; c += 16) {        // this half's D/2 columns
+          uint32_t o[16];
+          const uint32_t oc = tOx + half * (D / 2) + c;
+          tmem_load16(oc, o);
+          uint32_t o8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_store8(oc, o8);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[8 + i]) * alpha);
+          tmem_store8(oc + 8, o8);
+        }
+      }
       // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, partial row
       // sum; per 16 keys, their 16 score columns take 8 columns of hi weights
       // and (bf16) 8 of lo weights; one wait for all the stores
@@ -574,28 +592,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       tmem_store_wait();
       l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
-      // O is stable once the previous P.V is done; rescale this half's
-      // columns if the reference maximum moved
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, pf_wait(&o_done[x], (j - 1) & 1, abort, p.wait_ns));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, bump)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 2; c += 16) {        // this half's D/2 columns
-            uint32_t o[16];
-            const uint32_t oc = tOx + half * (D / 2) + c;
-            tmem_load16(oc, o);
-            uint32_t o8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_store8(oc, o8);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o8[i] = __float_as_uint(__uint_as_float(o[8 + i]) * alpha);
-            tmem_store8(oc + 8, o8);
-          }
-        }
-      }
       tc_fence_before();
       mbar_arrive(&p_full[x]);
     }
