@@ -214,3 +214,21 @@ def test_bf16_values_beyond_fp16_range_are_reported(pa, cuda_device):
     assert pa.pa_device_error() == pa.DEVERR["range"]
     rows0 = slice(int(b.query_start[0]), int(b.query_start[1]))
     assert max_abs_err(got[rows0], want[rows0]) <= TOL
+
+
+@pytest.mark.parametrize("S", [32, 40])
+def test_many_sequences_every_unit_runs(pa, cuda_device, S):
+    """Up to 32 sequences the launch order ranks them by context length (ties
+    by index), beyond that it keeps the plain order; either way every
+    (sequence, query-tile pair, kv head) unit runs: the output starts as NaN
+    and every row must match the oracle."""
+    rng = np.random.default_rng(100 + S)
+    sh = W.Shape(8, 2, 64, 16, "bf16")
+    lens = rng.integers(1, 600, size=S)
+    lens[::5] = 300                                   # tied context lengths
+    chunks = np.minimum(lens, rng.integers(1, 100, size=S))
+    b = W.make_prefill_batch(sh, lens, chunks, seed=S, device=cuda_device, poison="nan")
+    got, want = run_prefill(pa, b)
+    assert np.isfinite(got).all()
+    assert max_abs_err(got, want) <= TOL
+    assert pa.pa_device_error() == 0
