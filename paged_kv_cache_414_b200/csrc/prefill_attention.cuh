@@ -52,9 +52,8 @@
 //               than holding them).
 //
 // Tensor memory (512 columns): tile A's S at 0 and O at 128, tile B's S at
-// 256 and O at 384.  P replaces S in its own columns, 16 keys at a time: the
-// 16 columns holding those keys' scores take their 8 columns of fp16 weights
-// (two per column).  The MMA that next writes a tile's S columns is issued
+// 256 and O at 384.  P replaces S in its own columns: each key half's 64
+// fp16 weights (two per column) fill the first 32 of its 64 score columns.  The MMA that next writes a tile's S columns is issued
 // after that tile's P.V, and MMAs run in issue order.
 //
 // Every wait is bounded: on time-out a shared abort flag stops every role,
@@ -408,7 +407,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kPfKeys / 16; ++kk)   // 16 keys: 8 columns of P, 16 rows of V
-          umma_f16_ts(d, pj + kk * 16, dv + kk * ((16 * 128) >> 4), idO16, kk > 0 ? 1u : acc0);
+          umma_f16_ts(d, pj + (kk >> 2) * 64 + (kk & 3) * 8, dv + kk * ((16 * 128) >> 4), idO16,
+                      kk > 0 ? 1u : acc0);
         umma_commit(&o_done[x]);
       };
       bool ok = pf_wait(q_full, 0, abort, p.wait_ns) && pf_wait(&full_k[0], 0, abort, p.wait_ns);
@@ -564,21 +564,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tmem_store8(oc + 8, o8);
         }
       }
-      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory, partial row
-      // sum; per 16 keys, their 16 score columns take 8 columns of hi weights
-      // and (bf16) 8 of lo weights; one wait for all the stores
-      // (pairs of keys use packed two-lane fp32 instructions)
+      // pass 2: weights 2^(s*scale*log2e - m) -> tensor memory as fp16, and
+      // the partial row sum.  32 scores at a time are read, and their 32
+      // weights stored as 16 packed columns at the front of this half's
+      // columns (keys 32c .. 32c+31 at columns 16c .. 16c+15): a store only
+      // overwrites scores already read.  Pairs of keys use packed two-lane
+      // fp32 instructions; one wait for all the stores.
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t v[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if ((c & 1) == 0) tmem_load32(sj + c * 16, v);
-        uint32_t hp[8];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_load32(sj + c * 32, v);
+        uint32_t hp[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int k = c * 16 + 2 * i;
+        for (int i = 0; i < 16; ++i) {
+          const int k = c * 32 + 2 * i;
           float x0, x1;
-          ffma2(x0, x1, __uint_as_float(v[k & 31]), __uint_as_float(v[(k + 1) & 31]), sl2, sl2,
+          ffma2(x0, x1, __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]), sl2, sl2,
                 -m_new, -m_new);
           float p0 = fast_exp2(x0);
           float p1 = fast_exp2(x1);
@@ -588,7 +590,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           hp[i] = round_f16(p0, p1, &sum[(i & 1) * 2], &sum[(i & 1) * 2 + 1]);
         }
-        tmem_store8_async(sj + c * 16, hp);
+        tmem_store16_async(sj + c * 16, hp);
       }
       tmem_store_wait();
       l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
