@@ -74,8 +74,9 @@ typedef enum {
 #define PA_DEVERR_SLOT 0x4u        /* slot_mapping entry >= num_blocks * block_size */
 #define PA_DEVERR_COPY_PAIR 0x8u   /* copy_blocks pair outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x10u    /* a bounded wait on an asynchronous copy gave up */
-#define PA_DEVERR_RANGE 0x20u      /* prefill: a bf16 V value beyond fp16's range (|v| > 65504,
-                                      or not finite) was saturated */
+#define PA_DEVERR_RANGE 0x20u      /* prefill over a bf16 cache: an output row came out not
+                                      finite -- a V value beyond fp16's range (|v| >= 65520)
+                                      or a non-finite q, K or V element */
 
 /* Human-readable name of a pa_status value (static string). */
 const char *pa_status_string(int status);
@@ -292,8 +293,9 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
  * cache dtype; P.V in fp16 -- the softmax weights rounded to fp16 (2^-11
  * relative; the row sums add the rounded values), and a bf16 V tile converted
  * to fp16 in shared memory, which is exact for |v| <= 65504.  A bf16 V value
- * beyond that (or not finite) is saturated to fp16's largest value and sets
- * PA_DEVERR_RANGE: the rows attending to it are then inexact.  No workspace,
+ * of |v| >= 65520 becomes infinite there, so the output rows of the query tile
+ * that reads it come out not finite; PA_DEVERR_RANGE reports any non-finite
+ * output row of a bf16 cache (non-finite q or K elements included).  No workspace,
  * nothing allocated.  A chunk longer than its
  * context, a context longer than the table, or rows outside
  * [0, num_tokens) set PA_DEVERR_CONTEXT_LEN and leave that sequence's rows

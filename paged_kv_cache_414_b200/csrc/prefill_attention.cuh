@@ -23,7 +23,8 @@
 //               each lane issues one copy of a tile (one block, one 64-column
 //               chunk, K or V), and K and V land on separate barriers; K and V
 //               of a stage are released separately.
-//   warp 1      owns the tensor memory; one lane issues the MMAs, alternating
+//   warp 1      owns the tensor memory and issues the MMAs (the whole warp
+//               runs the loop, one elected lane issues), alternating
 //               between the query tiles so that one tile's MMAs run while the
 //               other tile's softmax does:
 //                 S_X = Q_X K_j^T   (M 128, N 128 keys, K = head_dim, cache dtype)
@@ -44,8 +45,10 @@
 //               tiles through shared memory and TMA stores.
 //   warps 18-21 V converter: zero the rows of a V tile past the last visible
 //               key and, for bf16 caches, rewrite the tile in place as fp16
-//               (exact for |v| <= 65504; saturated beyond, with
-//               PA_DEVERR_RANGE), so P.V is one fp16 MMA per 16 keys.  The
+//               (exact for |v| <= 65504; a value beyond fp16's range becomes
+//               infinite, the outputs it reaches come out non-finite, and the
+//               epilogue reports PA_DEVERR_RANGE), so P.V is one fp16 MMA per
+//               16 keys.  The
 //               conversion sits between a V tile's arrival and its P.V, so
 //               it gets four warps (at 704 threads every thread keeps 80
 //               registers: the softmax re-reads its scores from TMEM rather
@@ -168,13 +171,14 @@ __device__ __forceinline__ void fsub2(float &d0, float &d1, float a0, float a1, 
 }
 
 // A packed pair of bf16 values as a packed pair of fp16 values: exact within
-// fp16's range (bf16 has fewer significant bits), saturating beyond it; *big
-// keeps the largest magnitude seen.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x, float *big) {
+// fp16's range (bf16 has fewer significant bits); a value beyond it
+// (|v| >= 65520) becomes infinite.  No range test here: an infinite V makes
+// every output row of the tile that reads it non-finite, which the epilogue
+// checks once per row instead of once per element.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
   const float hi = __uint_as_float(x & 0xffff0000u), lo = __uint_as_float(x << 16);
-  *big = fmax3(*big, fabsf(hi), fabsf(lo));
   uint32_t y;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
   return y;
 }
 
@@ -376,14 +380,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
+    // (whole warp, warp-uniform waits; the wrappers elect the issuing lane)
+    {
       constexpr bool kBf = std::is_same<T, __nv_bfloat16>::value;
       const uint32_t idS = umma_idesc_f16(kBf, kPfRows, kPfKeys, false, false);
       const uint32_t idO16 = umma_idesc_f16(false, kPfRows, D, false, true);   // fp16 P and V
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
       // Shared-memory descriptors, built once: a k-step moves the start
       // address field by a constant, so every MMA below takes a
-      // precomputed base plus an immediate (the issuing thread shares its
+      // precomputed base plus an immediate (the issuing warp shares its
       // scheduler with softmax warps, so its instruction count per MMA is
       // what sets the issue rate).
       const uint64_t dQ0 = umma_desc_sw128(aQ, 16, 1024);
@@ -411,7 +416,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                       kk > 0 ? 1u : acc0);
         umma_commit(&o_done[x]);
       };
-      bool ok = pf_wait(q_full, 0, abort, p.wait_ns) && pf_wait(&full_k[0], 0, abort, p.wait_ns);
+      bool ok = __all_sync(0xffffffffu, pf_wait(q_full, 0, abort, p.wait_ns) &&
+                                            pf_wait(&full_k[0], 0, abort, p.wait_ns));
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -420,18 +426,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         // tile A: its P.V, then its next S (which overwrites its P, in issue order)
-        if (!pf_wait(&p_full[0], j & 1, abort, p.wait_ns)) break;
-        if (!pf_wait(&v_ready[j % NST], (j / NST) & 1, abort, p.wait_ns)) break;
+        if (!__all_sync(0xffffffffu, pf_wait(&p_full[0], j & 1, abort, p.wait_ns))) break;
+        if (!__all_sync(0xffffffffu, pf_wait(&v_ready[j % NST], (j / NST) & 1, abort, p.wait_ns))) break;
         tc_fence_after();
         issue_pv(0, j);
         const bool more = j + 1 < n_tiles;
         if (more) {
-          if (!pf_wait(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1, abort, p.wait_ns)) break;
+          if (!__all_sync(0xffffffffu, pf_wait(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1, abort, p.wait_ns))) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
         // tile B
-        if (!pf_wait(&p_full[1], j & 1, abort, p.wait_ns)) break;
+        if (!__all_sync(0xffffffffu, pf_wait(&p_full[1], j & 1, abort, p.wait_ns))) break;
         tc_fence_after();
         issue_pv(1, j);
         umma_commit(&empty_v[j % NST]);
@@ -448,13 +454,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // Each landed V tile, before its P.V: rows past the last visible key are
     // zeroed (masked for every row, but 0 x NaN from stale or poisoned bits
     // would reach O), and a bf16 tile is rewritten in place as fp16 -- exact
-    // for |v| <= 65504, fp16's largest value; beyond it the value saturates
-    // there and PA_DEVERR_RANGE is set -- so that P.V takes one fp16 P.  An
-    // element keeps its byte position, so the swizzle is untouched.
+    // for |v| <= 65504, fp16's largest value; beyond it the value becomes
+    // infinite and the epilogue reports the non-finite rows -- so that P.V
+    // takes one fp16 P.  An element keeps its byte position, so the swizzle
+    // is untouched.  The conversion's instruction count matters: these warps
+    // share their schedulers with the softmax.
     const int ct = threadIdx.x - 18 * 32;          // 0 .. 127
     constexpr int NCHUNK = NCH * kPfKeys * 8;      // 16-byte chunks of a V tile
     constexpr bool kBf = std::is_same<T, __nv_bfloat16>::value;
-    float big = 0.f;                               // largest |v| of the bf16 values kept
     for (int j = 0; j < n_tiles; ++j) {
       const int st = j % NST;
       if (!__all_sync(0xffffffffu, pf_wait(&full_v[st], (j / NST) & 1, abort, p.wait_ns)))
@@ -467,15 +474,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           *c = make_uint4(0, 0, 0, 0);
         } else if (kBf) {
           const uint4 w = *c;
-          *c = make_uint4(bf16x2_to_f16x2(w.x, &big), bf16x2_to_f16x2(w.y, &big),
-                          bf16x2_to_f16x2(w.z, &big), bf16x2_to_f16x2(w.w, &big));
+          *c = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z),
+                          bf16x2_to_f16x2(w.w));
         }
       }
       // generic-proxy writes, read next by the tensor cores (async proxy)
       fence_proxy_async_smem();
       mbar_arrive(&v_ready[st]);
     }
-    if (kBf && !(big <= 65504.f)) flag_error(PA_DEVERR_RANGE);   // beyond fp16, or infinite
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int x = (warp - 2) >> 3;                // query tile: warps 2-9 A, 10-17 B
@@ -614,6 +620,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const bool full_tile = tokx + p.tq <= C;
     uint8_t *ostage = x == 0 ? sK : sV;
     constexpr int OBOX = kPfRows * 128;           // one 32-column box of 128 rows
+    float fin = 0.f;                              // sum of this thread's outputs
     if (ok) {
       tc_fence_after();
       l += *reinterpret_cast<volatile float *>(slot(2, 1 - half));
@@ -631,6 +638,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const float4 val =
               make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
                           __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          if (row_ok) fin += (val.x + val.y) + (val.z + val.w);
           if (full_tile) {
             const int chunk = ((col0 & 31) + i) >> 2;   // 16-byte chunk within the box row
             *reinterpret_cast<float4 *>(box + ((chunk ^ (r & 7)) << 4)) = val;
@@ -640,6 +648,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
     }
+    // A bf16 V value beyond fp16's range became infinite in the P.V (and a
+    // non-finite q or K gives non-finite scores): the row's outputs are then
+    // not finite, and so is their sum (the outputs of finite inputs are
+    // bounded by max |v|, far from overflowing it).
+    if (std::is_same<T, __nv_bfloat16>::value && !(fabsf(fin) <= 3.0e38f))
+      flag_error(PA_DEVERR_RANGE);
     if (full_tile) {
       // every thread of the tile reaches this barrier, whether or not it
       // aborted: the branch above holds no early exit

@@ -203,9 +203,9 @@ def test_bad_block_id_reports_instead_of_faulting(pa, cuda_device):
 
 def test_bf16_values_beyond_fp16_range_are_reported(pa, cuda_device):
     """P.V runs in fp16, with a bf16 V tile converted exactly within fp16's
-    range; a bf16 V value beyond it is saturated and reported
-    (PA_DEVERR_RANGE), never silent.  Sequences that never read the value
-    still match the oracle."""
+    range; a bf16 V value beyond it becomes infinite, the rows that read it
+    come out not finite, and that is reported (PA_DEVERR_RANGE), never
+    silent.  Sequences that never read the value still match the oracle."""
     sh = W.Shape(8, 2, 128, 16, "bf16")
     b = W.make_prefill_batch(sh, [300, 500], [100, 200], seed=9, device=cuda_device)
     blk = int(b.block_tables[1, 0])                  # a prefix block of sequence 1
@@ -214,6 +214,22 @@ def test_bf16_values_beyond_fp16_range_are_reported(pa, cuda_device):
     assert pa.pa_device_error() == pa.DEVERR["range"]
     rows0 = slice(int(b.query_start[0]), int(b.query_start[1]))
     assert max_abs_err(got[rows0], want[rows0]) <= TOL
+    rows1 = slice(int(b.query_start[1]), int(b.query_start[2]))
+    assert not np.isfinite(got[rows1, 0:4]).all()     # kv head 0's query heads
+
+
+def test_finite_bf16_inputs_raise_no_range_flag(pa, cuda_device):
+    """The range check looks at the outputs: large finite V values inside
+    fp16's range (65280, bf16's largest below 65504) convert exactly and are
+    not reported."""
+    sh = W.Shape(8, 2, 128, 16, "bf16")
+    b = W.make_prefill_batch(sh, [300, 500], [100, 200], seed=19, device=cuda_device)
+    blk = int(b.block_tables[1, 0])
+    b.v_cache[blk, 0, 3, 5] = 65280.0
+    b.v_cache[blk, 1, 7, 9] = -65280.0
+    got, want = run_prefill(pa, b)
+    assert pa.pa_device_error() == 0
+    assert max_abs_err(got, want) <= TOL * 65280.0
 
 
 @pytest.mark.parametrize("S", [32, 40])
