@@ -43,16 +43,15 @@
 //               O is rescaled in tensor memory when the row maximum moves by
 //               more than 2^8; the epilogue writes out = O / l, full query
 //               tiles through shared memory and TMA stores.
-//   warps 18-21 V converter: zero the rows of a V tile past the last visible
+//   warps 18-23 V converter: zero the rows of a V tile past the last visible
 //               key and, for bf16 caches, rewrite the tile in place as fp16
 //               (exact for |v| <= 65504; a value beyond fp16's range becomes
 //               infinite, the outputs it reaches come out non-finite, and the
 //               epilogue reports PA_DEVERR_RANGE), so P.V is one fp16 MMA per
-//               16 keys.  The
-//               conversion sits between a V tile's arrival and its P.V, so
-//               it gets four warps (at 704 threads every thread keeps 80
-//               registers: the softmax re-reads its scores from TMEM rather
-//               than holding them).
+//               16 keys.  The conversion sits between a V tile's arrival and
+//               its P.V, so it gets six warps (at 768 threads every thread
+//               keeps 80 registers: the softmax re-reads its scores from TMEM
+//               rather than holding them).
 //
 // Tensor memory (512 columns): tile A's S at 0 and O at 128, tile B's S at
 // 256 and O at 384.  P replaces S in its own columns: each key half's 64
@@ -87,7 +86,8 @@ struct PrefillParams {
 
 constexpr int kPfRows = 128;      // query rows per query tile
 constexpr int kPfKeys = 128;      // keys per K/V tile
-constexpr int kPfThreads = 704;   // producer, MMA, 2 x 8 softmax warps, 4 V-converter warps
+constexpr int kPfThreads = 768;   // producer, MMA, 2 x 8 softmax warps, 6 V-converter warps
+constexpr int kPfConv = 192;      // V-converter threads
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint64_t kPfDrainLimitNs = 2000000000ull;   // draining after an abort
 
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&full_v[i], 1);
       mbar_init(&empty_k[i], 1);
       mbar_init(&empty_v[i], 1);
-      mbar_init(&v_ready[i], 128);
+      mbar_init(&v_ready[i], kPfConv);
     }
 
     mbar_init(q_full, 1);
@@ -398,22 +398,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       auto issue_s = [&](int x, int j) {        // S_x = Q_x K_j^T
         const uint64_t dq = dQ0 + x * kQStep, dk = dK0 + (j % NST) * kStageStep;
         const uint32_t d = tmem + x * 256;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          constexpr uint32_t kRegion = L::REGION >> 4;
-          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 2;
-          umma_f16_ss(d, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
-        }
+        constexpr uint32_t kRegion = L::REGION >> 4;
+        if constexpr (D == 128)
+          umma_ss_group8<0, 2, 4, 6, kRegion, kRegion + 2, kRegion + 4, kRegion + 6>(d, dq, dk, idS, 0u);
+        else
+          umma_ss_group4<0, 2, 4, 6>(d, dq, dk, idS, 0u);
         umma_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {       // O_x += P_x V_j, fp16 P and V
         const uint64_t dv = dV0 + (j % NST) * kStageStep;
         const uint32_t pj = tmem + x * 256, d = pj + 128;
         const uint32_t acc0 = j > 0 ? 1u : 0u;
-#pragma unroll
-        for (int kk = 0; kk < kPfKeys / 16; ++kk)   // 16 keys: 8 columns of P, 16 rows of V
-          umma_f16_ts(d, pj + (kk >> 2) * 64 + (kk & 3) * 8, dv + kk * ((16 * 128) >> 4), idO16,
-                      kk > 0 ? 1u : acc0);
+        // 16 keys per step: 8 columns of P, 16 rows of V
+        umma_ts_group8<0, 8, 16, 24, 64, 72, 80, 88, 0, 128, 256, 384, 512, 640, 768, 896>(
+            d, pj, dv, idO16, acc0);
         umma_commit(&o_done[x]);
       };
       bool ok = __all_sync(0xffffffffu, pf_wait(q_full, 0, abort, p.wait_ns) &&
@@ -459,7 +457,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // takes one fp16 P.  An element keeps its byte position, so the swizzle
     // is untouched.  The conversion's instruction count matters: these warps
     // share their schedulers with the softmax.
-    const int ct = threadIdx.x - 18 * 32;          // 0 .. 127
+    const int ct = threadIdx.x - 18 * 32;          // 0 .. kPfConv - 1
     constexpr int NCHUNK = NCH * kPfKeys * 8;      // 16-byte chunks of a V tile
     constexpr bool kBf = std::is_same<T, __nv_bfloat16>::value;
     for (int j = 0; j < n_tiles; ++j) {
@@ -468,7 +466,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         break;
       uint8_t *v0 = sV + st * L::KV_BYTES;
       const int z0 = j == n_tiles - 1 ? pos_max + 1 - j * kPfKeys : kPfKeys;   // first dead row
-      for (int i = ct; i < NCHUNK; i += 128) {
+      for (int i = ct; i < NCHUNK; i += kPfConv) {
         uint4 *c = reinterpret_cast<uint4 *>(v0 + i * 16);
         if (((i >> 3) & (kPfKeys - 1)) >= z0) {
           *c = make_uint4(0, 0, 0, 0);

@@ -76,36 +76,82 @@ __device__ __forceinline__ void tc_fence_after() {
 
 // The MMA and commit wrappers below are executed by a whole warp with
 // warp-uniform operands; one lane, chosen by elect.sync, issues the
-// instruction.  Keeping the issuing code warp-uniform lets the compiler hold
+// instructions (a fully active warp always elects the same lane, so commits
+// track every MMA of the warp).  Keeping the issuing code warp-uniform lets the compiler hold
 // the descriptors in uniform registers instead of moving them there before
 // every MMA, which measurably speeds up issue when the issuing warp shares
 // its scheduler with busy warps.
 
-// D[tmem] = A * B (+ D when `accumulate`), A and B described in shared memory.
-__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+// Groups of MMAs in one statement: one elect and one predicate set-up for
+// all of them, each step's descriptors the group's base plus an immediate
+// added to the low word (the start-address field, 16-byte units; bases and
+// offsets keep it inside its 14 bits).  The first step accumulates into D
+// when acc0 != 0, the others always.  Operands: %0 D (TMEM), %1 A, %2 B,
+// %3 instruction descriptor, %4 acc0, then the step offsets.
+
+// One step with A and B in shared memory, both moved by operand OP.
+#define PA_UMMA_SS_STEP(OP, PRED)                                               \
+  "add.u32 al, a0, %" #OP ";\n\tadd.u32 bl, b0, %" #OP ";\n\t"                  \
+  "mov.b64 da, {al, ah};\n\tmov.b64 db, {bl, bh};\n\t"                          \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, " PRED ";\n\t"
+// One step with A in tensor memory (column offset operand OA) and B in shared
+// memory (start-address offset operand OB).
+#define PA_UMMA_TS_STEP(OA, OB, PRED)                                           \
+  "add.u32 at, %1, %" #OA ";\n\tadd.u32 bl, b0, %" #OB ";\n\t"                  \
+  "mov.b64 db, {bl, bh};\n\t"                                                   \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [at], db, %3, " PRED ";\n\t"
+#define PA_UMMA_GROUP_HEAD                                                      \
+  "{\n\t.reg .pred e, p, t;\n\t.reg .b32 a0, ah, b0, bh, al, bl, at;\n\t"       \
+  ".reg .b64 da, db;\n\t"                                                       \
+  "elect.sync _|e, 0xffffffff;\n\t"                                             \
+  "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"                          \
+  "mov.b64 {b0, bh}, %2;\n\t"
+
+// Eight kind::f16 steps, A and B in shared memory, both moved by O0..O7.
+template <uint32_t O0, uint32_t O1, uint32_t O2, uint32_t O3, uint32_t O4, uint32_t O5,
+          uint32_t O6, uint32_t O7>
+__device__ __forceinline__ void umma_ss_group8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t acc0) {
+  asm volatile(PA_UMMA_GROUP_HEAD "mov.b64 {a0, ah}, %1;\n\t"
+               PA_UMMA_SS_STEP(5, "p") PA_UMMA_SS_STEP(6, "t") PA_UMMA_SS_STEP(7, "t")
+               PA_UMMA_SS_STEP(8, "t") PA_UMMA_SS_STEP(9, "t") PA_UMMA_SS_STEP(10, "t")
+               PA_UMMA_SS_STEP(11, "t") PA_UMMA_SS_STEP(12, "t") "}" ::"r"(d),
+               "l"(a), "l"(b), "r"(idesc), "r"(acc0), "n"(O0), "n"(O1), "n"(O2), "n"(O3),
+               "n"(O4), "n"(O5), "n"(O6), "n"(O7)
+               : "memory");
 }
 
-// D[tmem] = A * B (+ D when `accumulate`), A in tensor memory (row i of A in
-// lane i, two 16-bit elements per 32-bit column, the lower index in the low
-// half), B described in shared memory.
-__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+// Four such steps.
+template <uint32_t O0, uint32_t O1, uint32_t O2, uint32_t O3>
+__device__ __forceinline__ void umma_ss_group4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t acc0) {
+  asm volatile(PA_UMMA_GROUP_HEAD "mov.b64 {a0, ah}, %1;\n\t"
+               PA_UMMA_SS_STEP(5, "p") PA_UMMA_SS_STEP(6, "t") PA_UMMA_SS_STEP(7, "t")
+               PA_UMMA_SS_STEP(8, "t") "}" ::"r"(d),
+               "l"(a), "l"(b), "r"(idesc), "r"(acc0), "n"(O0), "n"(O1), "n"(O2), "n"(O3)
+               : "memory");
 }
+
+// Eight steps with A in tensor memory (column offsets A0..A7 from a_tmem) and
+// B in shared memory (start-address offsets B0..B7).
+template <uint32_t A0, uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5,
+          uint32_t A6, uint32_t A7, uint32_t B0, uint32_t B1, uint32_t B2, uint32_t B3,
+          uint32_t B4, uint32_t B5, uint32_t B6, uint32_t B7>
+__device__ __forceinline__ void umma_ts_group8(uint32_t d, uint32_t a_tmem, uint64_t b,
+                                               uint32_t idesc, uint32_t acc0) {
+  asm volatile(PA_UMMA_GROUP_HEAD
+               PA_UMMA_TS_STEP(5, 13, "p") PA_UMMA_TS_STEP(6, 14, "t") PA_UMMA_TS_STEP(7, 15, "t")
+               PA_UMMA_TS_STEP(8, 16, "t") PA_UMMA_TS_STEP(9, 17, "t") PA_UMMA_TS_STEP(10, 18, "t")
+               PA_UMMA_TS_STEP(11, 19, "t") PA_UMMA_TS_STEP(12, 20, "t") "}" ::"r"(d),
+               "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc0), "n"(A0), "n"(A1), "n"(A2), "n"(A3),
+               "n"(A4), "n"(A5), "n"(A6), "n"(A7), "n"(B0), "n"(B1), "n"(B2), "n"(B3), "n"(B4),
+               "n"(B5), "n"(B6), "n"(B7)
+               : "memory");
+}
+
+#undef PA_UMMA_SS_STEP
+#undef PA_UMMA_TS_STEP
+#undef PA_UMMA_GROUP_HEAD
 
 // Arrive once on `bar` when every MMA the warp issued before has completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
