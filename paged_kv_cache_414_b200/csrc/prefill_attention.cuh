@@ -662,7 +662,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int b = 0; b < D / 32; ++b)
           tma_store_3d(&omap, ostage + b * OBOX, b * 32, kh * G, q0 + tokx);
         bulk_commit_group();
-        bulk_wait_group0();
+        bulk_wait_group_read0();     // the ring is free once the stores read it
       }
     }
   }

@@ -253,10 +253,11 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void 
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// Wait until every bulk store this thread committed has completed (its
-// shared-memory source is free and its global writes are done).
-__device__ __forceinline__ void bulk_wait_group0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+// Wait until every bulk store this thread committed has read its
+// shared-memory source (which may then be reused or freed; the global
+// writes complete on their own, before the grid counts as finished).
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // Barrier among `count` threads of the CTA on hardware barrier `id` (1..15).
