@@ -55,8 +55,9 @@
 //
 // Tensor memory (512 columns): tile A's S at 0 and O at 128, tile B's S at
 // 256 and O at 384.  P replaces S in its own columns: each key half's 64
-// fp16 weights (two per column) fill the first 32 of its 64 score columns.  The MMA that next writes a tile's S columns is issued
-// after that tile's P.V, and MMAs run in issue order.
+// fp16 weights (two per column) fill the first 32 of its 64 score columns.
+// The MMA that next writes a tile's S columns is issued after that tile's
+// P.V, and MMAs run in issue order.
 //
 // Every wait is bounded: on time-out a shared abort flag stops every role,
 // PA_DEVERR_TIMEOUT is set, copies and MMAs in flight are waited for (again
@@ -354,7 +355,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int off = st * L::KV_BYTES + cc * kPfKeys * 128 + cb * B * 128;
       const int row = (id * p.num_kv_heads + kh) * B;
       if (j >= NST) {
-        const bool w = lane == 0 ? pf_wait(&empty_k[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
+        const bool w =
+            lane == 0 ? pf_wait(&empty_k[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
         if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
       if (lane == 0) mbar_arrive_expect_tx(&full_k[st], __popc(valid & 0x55555555u) * B * 128);
@@ -362,7 +364,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (id >= 0 && ckv == 0) tma_load_2d(sK + off, &kmap, cc * 64, row, &full_k[st]);
       issued_k = j + 1;
       if (j >= NST) {
-        const bool w = lane == 0 ? pf_wait(&empty_v[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
+        const bool w =
+            lane == 0 ? pf_wait(&empty_v[st], (j / NST - 1) & 1, abort, p.wait_ns) : true;
         if (!__shfl_sync(0xffffffffu, w, 0)) break;
       }
       if (lane == 0) mbar_arrive_expect_tx(&full_v[st], __popc(valid & 0xAAAAAAAAu) * B * 128);
@@ -400,7 +403,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t d = tmem + x * 256;
         constexpr uint32_t kRegion = L::REGION >> 4;
         if constexpr (D == 128)
-          umma_ss_group8<0, 2, 4, 6, kRegion, kRegion + 2, kRegion + 4, kRegion + 6>(d, dq, dk, idS, 0u);
+          umma_ss_group8<0, 2, 4, 6, kRegion, kRegion + 2, kRegion + 4, kRegion + 6>(d, dq, dk,
+                                                                                      idS, 0u);
         else
           umma_ss_group4<0, 2, 4, 6>(d, dq, dk, idS, 0u);
         umma_commit(&s_full[x]);
@@ -414,8 +418,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             d, pj, dv, idO16, acc0);
         umma_commit(&o_done[x]);
       };
-      bool ok = __all_sync(0xffffffffu, pf_wait(q_full, 0, abort, p.wait_ns) &&
-                                            pf_wait(&full_k[0], 0, abort, p.wait_ns));
+      // every lane waits; the warp goes on only if all of them saw the phase
+      auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, pf_wait(bar, parity, abort, p.wait_ns));
+      };
+      bool ok = wait_all(q_full, 0) && wait_all(&full_k[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -424,18 +431,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         // tile A: its P.V, then its next S (which overwrites its P, in issue order)
-        if (!__all_sync(0xffffffffu, pf_wait(&p_full[0], j & 1, abort, p.wait_ns))) break;
-        if (!__all_sync(0xffffffffu, pf_wait(&v_ready[j % NST], (j / NST) & 1, abort, p.wait_ns))) break;
+        if (!wait_all(&p_full[0], j & 1)) break;
+        if (!wait_all(&v_ready[j % NST], (j / NST) & 1)) break;
         tc_fence_after();
         issue_pv(0, j);
         const bool more = j + 1 < n_tiles;
         if (more) {
-          if (!__all_sync(0xffffffffu, pf_wait(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1, abort, p.wait_ns))) break;
+          if (!wait_all(&full_k[(j + 1) % NST], ((j + 1) / NST) & 1)) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
         // tile B
-        if (!__all_sync(0xffffffffu, pf_wait(&p_full[1], j & 1, abort, p.wait_ns))) break;
+        if (!wait_all(&p_full[1], j & 1)) break;
         tc_fence_after();
         issue_pv(1, j);
         umma_commit(&empty_v[j % NST]);

@@ -77,10 +77,10 @@ __device__ __forceinline__ void tc_fence_after() {
 // The MMA and commit wrappers below are executed by a whole warp with
 // warp-uniform operands; one lane, chosen by elect.sync, issues the
 // instructions (a fully active warp always elects the same lane, so commits
-// track every MMA of the warp).  Keeping the issuing code warp-uniform lets the compiler hold
-// the descriptors in uniform registers instead of moving them there before
-// every MMA, which measurably speeds up issue when the issuing warp shares
-// its scheduler with busy warps.
+// track every MMA of the warp).  Keeping the issuing code warp-uniform lets
+// the compiler hold the descriptors in uniform registers instead of moving
+// them there before every MMA, which measurably speeds up issue when the
+// issuing warp shares its scheduler with busy warps.
 
 // Groups of MMAs in one statement: one elect and one predicate set-up for
 // all of them, each step's descriptors the group's base plus an immediate
@@ -132,8 +132,9 @@ __device__ __forceinline__ void umma_ss_group4(uint32_t d, uint64_t a, uint64_t 
                : "memory");
 }
 
-// Eight steps with A in tensor memory (column offsets A0..A7 from a_tmem) and
-// B in shared memory (start-address offsets B0..B7).
+// Eight steps with A in tensor memory (column offsets A0..A7 from a_tmem; row
+// i of A in lane i, two 16-bit elements per 32-bit column, the lower index in
+// the low half) and B in shared memory (start-address offsets B0..B7).
 template <uint32_t A0, uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5,
           uint32_t A6, uint32_t A7, uint32_t B0, uint32_t B1, uint32_t B2, uint32_t B3,
           uint32_t B4, uint32_t B5, uint32_t B6, uint32_t B7>
